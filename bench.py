@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the MLA hot path on B200: one step = one DeepSeek-V3-shaped
+prefill forward (B=1, T=4096, hidden 7168, 128 heads, YaRN) followed by one
+weight-absorbed decode step (B=64, context lengths uniform in [1024, 32768]).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  ``value`` is the prefill throughput in
+TFLOP/s (algorithmic FLOPs of the forward, causal attention counted for
+j <= i only) over all ranks; decode latent-cache GB/s and prefill tokens/s are
+reported beside it.  Multi-GPU runs are independent replicas (weak scaling,
+no collective on the data path); the timing is the max over ranks.
+"""
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "dsv3_prefill"
+DECODE = "dsv3_decode"
+L2_FLUSH_BYTES = 256 << 20
+STAGES_P = ["s1_down_proj", "s3_q_proj", "s4_kv_up_proj", "s7_attention",
+            "s8_o_proj"]
+STAGES_D = ["d1_q_absorb", "d2_latent_attention", "d3_combine", "d4_v_up",
+            "o_proj"]
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work
+# ---------------------------------------------------------------------------
+def prefill_stage_flops(cfg, B, T):
+    N = B * T
+    H, h = cfg.hidden_size, cfg.num_heads
+    dn, dr, dv = cfg.qk_nope_head_dim, cfg.qk_rope_head_dim, cfg.v_head_dim
+    dq, rq, rkv = dn + dr, cfg.q_lora_rank, cfg.kv_lora_rank
+    down = 2 * N * H * ((rq if rq else 0) + rkv + dr)
+    q = 2 * N * (rq * h * dq if rq else H * h * dq)
+    kv = 2 * N * rkv * h * (dn + dv)
+    attn = B * h * (dq + dv) * T * (T + 1)          # 2 FLOP x causal pairs
+    o = 2 * N * h * dv * H
+    return {"s1_down_proj": down, "s3_q_proj": q, "s4_kv_up_proj": kv,
+            "s7_attention": attn, "s8_o_proj": o}
+
+
+def decode_work(cfg, ctx_total, B):
+    h, r, dr, dn, dv = (cfg.num_heads, cfg.kv_lora_rank, cfg.qk_rope_head_dim,
+                        cfg.qk_nope_head_dim, cfg.v_head_dim)
+    cache_bytes = ctx_total * (r + dr) * 2
+    wkvb = h * (dn + dv) * r * 2
+    qio = B * h * (dn + dr) * 2 + B * h * dv * 2
+    flops = ctx_total * h * 2 * ((r + dr) + r) + 2 * B * h * r * (dn + dv)
+    return {"cache_bytes": cache_bytes, "bytes": cache_bytes + wkvb + qio,
+            "flops": flops}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "latent_attention_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def load_traffic():
+    """ncu DRAM bytes per launch, valid only for the sources they were taken on."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    d = json.load(open(p))
+    if d.get("source_hash") != source_hash():
+        return {}
+    return d.get("per_launch_bytes", {})
+
+
+# ---------------------------------------------------------------------------
+# Clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for l in self.lines:
+            p = [x.strip() for x in l.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx = float(p[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return local_rank
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_prefill_sample(cfg, inp, rows):
+    """Time the fp64 oracle on keys/values for all T positions plus the query
+    path, attention and o_proj for ``rows``; returns (seconds, FLOPs done)."""
+    import oracle
+    import numpy as np
+    t0 = time.perf_counter()
+    oracle.prefill(cfg, inp, rows=rows)
+    dt = time.perf_counter() - t0
+    B, T = inp.B, inp.T
+    R = len(rows)
+    f = prefill_stage_flops(cfg, B, T)
+    N = B * T
+    H, h = cfg.hidden_size, cfg.num_heads
+    dq, dv = cfg.qk_head_dim, cfg.v_head_dim
+    done = (2 * N * H * (cfg.kv_lora_rank + cfg.qk_rope_head_dim) +
+            f["s4_kv_up_proj"] +
+            (f["s1_down_proj"] - 2 * N * H * (cfg.kv_lora_rank + cfg.qk_rope_head_dim)) * R / T +
+            f["s3_q_proj"] * R / T +
+            B * h * (dq + dv) * 2 * float(np.sum(np.asarray(rows) + 1)) +
+            f["s8_o_proj"] * R / T)
+    return dt, done
+
+
+def cpu_threads():
+    try:
+        import torch
+        return torch.get_num_threads()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    from mla_inputs import WORKLOADS, make_prefill_inputs
+    wl = WORKLOADS[PREFILL]
+    inp = make_prefill_inputs(wl.cfg, wl.batch, wl.seq_len, seed=0)
+    rows = [0, 1, wl.seq_len // 2, wl.seq_len - 1]
+    secs, flops = [], 0.0
+    for i in range(args.warmup + args.steps):
+        dt, fl = oracle_prefill_sample(wl.cfg, inp, rows)
+        if i >= args.warmup:
+            secs.append(dt)
+            flops = fl
+    tot = sum(secs)
+    v = flops * len(secs) / tot / 1e12
+    sample = (f"fp64 NumPy oracle, {wl.name}: keys/values for all {wl.seq_len} "
+              f"positions + query/attention/o_proj for rows {rows}")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / len(secs), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_block(wl, None),
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "MLA prefill TFLOP/s + tokens/s; absorbed-decode latent-cache HBM GB/s"
+
+
+def config_block(wl, dwl):
+    c = wl.cfg
+    d = {"workload": f"{wl.name} (B={wl.batch}, T={wl.seq_len}) + "
+                     f"{DECODE} (B=64, ctx U[1024,32768])",
+         "prefill": {"B": wl.batch, "T": wl.seq_len, "hidden": c.hidden_size,
+                     "heads": c.num_heads, "q_lora_rank": c.q_lora_rank,
+                     "kv_lora_rank": c.kv_lora_rank, "qk_nope": c.qk_nope_head_dim,
+                     "qk_rope": c.qk_rope_head_dim, "v_head": c.v_head_dim,
+                     "rope": f"{c.rope_type} factor {c.rope_factor}"},
+         "l2": "flushed between steps (256 MiB write)",
+         "parallelism": "independent replicas, one per GPU"}
+    if dwl is not None:
+        d["decode"] = dwl
+    return d
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import torch
+    import torch.distributed as dist
+    import ctypes as C
+    from datetime import timedelta
+    from mla_inputs import (WORKLOADS, make_prefill_inputs, make_decode_inputs,
+                            decode_context_lengths)
+    import latent_attention_b200 as L
+    from latent_attention_b200 import _lib
+    from latent_attention_b200.layer import MlaPrefill, MlaDecode
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    lib = _lib.load()
+
+    wl, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+    cfg, cfgd = wl.cfg, wd.cfg
+    B, T = wl.batch, wl.seq_len
+    inp = make_prefill_inputs(cfg, B, T, seed=1000 * rank)
+    weights = {k: getattr(inp, k) for k in ("w_q_a", "g_q_a", "w_q_b", "w_q",
+                                              "w_kv_a", "g_kv_a", "w_kv_b", "w_o")}
+    pre = MlaPrefill(cfg, weights, B, T, device=dev)
+    x = inp.x.to(dev)
+    out = torch.empty(B, T, cfg.hidden_size, dtype=torch.bfloat16, device=dev)
+
+    ctx = decode_context_lengths(wd.batch, wd.ctx_min, wd.ctx_max, seed=rank)
+    di = make_decode_inputs(cfgd, wd.batch, ctx, seed=1000 * rank + 1)
+    dec = MlaDecode(cfgd, wd.batch, wd.ctx_max, device=dev)
+    qn, qp = di.q_nope.to(dev), di.q_pe.to(dev)
+    wkvb, cache, cu = di.w_kv_b.to(dev), di.cache.to(dev), di.cu_ctx.to(dev)
+    dout = torch.empty(wd.batch, cfgd.num_heads * cfgd.v_head_dim,
+                       dtype=torch.bfloat16, device=dev)
+    ctx_total = int(ctx.sum())
+    del inp, di
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    K, Wm = args.steps, args.warmup
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev_p = [[mk() for _ in range(6)] for _ in range(K)]
+    ev_d = [[mk() for _ in range(6)] for _ in range(K)]
+    ev_s = [(mk(), mk()) for _ in range(K)]
+
+    def set_events(evs):
+        if evs is None:
+            lib.mla_set_stage_events(None, 0)
+            return
+        arr = (C.c_void_p * len(evs))(*[e.cuda_event for e in evs])
+        lib.mla_set_stage_events(arr, len(evs))
+
+    def step(i):
+        timed = i >= Wm
+        j = i - Wm
+        if timed:
+            ev_s[j][0].record()
+        set_events(ev_p[j] if timed else None)
+        pre(x, out=out)
+        set_events(ev_d[j] if timed else None)
+        dec(qn, qp, wkvb, cache, cu, dout)
+        set_events(None)
+        if timed:
+            ev_s[j][1].record()
+
+    clocks = ClockSampler(gpu_index(local))
+    launches0 = 0
+    for i in range(Wm + K):
+        flush.zero_()
+        if i == Wm:
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            clocks.start()
+            launches0 = lib.mla_kernel_launches()
+        step(i)
+    torch.cuda.synchronize()
+    launches = lib.mla_kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    pre.check_status()
+    dec.check_status()
+
+    step_ms = sum(a.elapsed_time(b) for a, b in ev_s)
+    pre_ms = sum(e[0].elapsed_time(e[5]) for e in ev_p)
+    dec_ms = sum(e[0].elapsed_time(e[5]) for e in ev_d)
+    st_p = {n: sum(e[k].elapsed_time(e[k + 1]) for e in ev_p) / K
+            for k, n in enumerate(STAGES_P)}
+    st_d = {n: sum(e[k].elapsed_time(e[k + 1]) for e in ev_d) / K
+            for k, n in enumerate(STAGES_D)}
+    t = torch.tensor([step_ms, pre_ms, dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, pre_ms, dec_ms = t.tolist()
+
+    # ---- end to end through the public API with host buffers -------------
+    x_h = torch.empty_like(x, device="cpu").pin_memory()
+    x_h.copy_(x.cpu())
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    e2e_ev = [(mk(), mk()) for _ in range(K)]
+    for i in range(Wm + K):
+        flush.zero_()
+        if i >= Wm:
+            e2e_ev[i - Wm][0].record()
+        x.copy_(x_h, non_blocking=True)
+        pre(x, out=out)
+        out_h.copy_(out, non_blocking=True)
+        if i >= Wm:
+            e2e_ev[i - Wm][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev)],
+                          dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    fl = prefill_stage_flops(cfg, B, T)
+    pflops = sum(fl.values())
+    dw = decode_work(cfgd, ctx_total, wd.batch)
+    peaks = load_peaks()
+    traffic = load_traffic()
+    value = world * K * pflops / (pre_ms * 1e-3) / 1e12
+
+    def roof(stage, ms, bound):
+        if bound == "tensor":
+            a = fl[stage] / (ms * 1e-3) / 1e12
+            return {"bound": "tensor", "achieved": a, "peak": peaks["bf16_sustained"],
+                    "unit": "TFLOP/s", "frac": a / peaks["bf16_sustained"],
+                    "traffic": traffic.get(stage)}
+        a = dw["bytes"] / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": a, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": a / peaks["hbm"], "traffic": traffic.get(stage)}
+
+    stages = {n: roof(n, st_p[n], "tensor") for n in STAGES_P}
+    stages["d2_latent_attention"] = roof("d2_latent_attention",
+                                         st_d["d2_latent_attention"], "hbm")
+    dominant = max(STAGES_P, key=lambda n: st_p[n])
+    roofline = dict(stages[dominant], kernel=dominant,
+                    peak_source=f"{peaks['source']} (bf16 sustained / HBM copy)")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from mla_inputs import make_prefill_inputs as mpi
+        inp_c = mpi(cfg, B, T, seed=0)
+        rows = list(range(0, 8)) + list(range(T - 8, T))
+        dt, done = oracle_prefill_sample(cfg, inp_c, rows)
+        cpu = {"value": done / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+               "kind": "oracle",
+               "sample": f"fp64 NumPy oracle on {PREFILL}: keys/values for all {T} "
+                         f"positions + query/attention/o_proj for 16 rows "
+                         f"({done / 1e9:.0f} GFLOP in {dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K, "warmup": Wm, "ms_per_step": step_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded; random-init weights of "
+                                     "the DeepSeek-V3 MLA layer shapes)",
+            "config": config_block(wl, {"B": wd.batch, "ctx_total": ctx_total,
+                                        "ctx_range": [wd.ctx_min, wd.ctx_max]}),
+            "prefill_ms": pre_ms / K,
+            "prefill_tokens_per_s": world * K * B * T / (pre_ms * 1e-3),
+            "decode_ms": dec_ms / K,
+            "decode_latent_cache_gb_per_s": world * K * dw["cache_bytes"] / (dec_ms * 1e-3) / 1e9,
+            "decode_tflops": world * K * dw["flops"] / (dec_ms * 1e-3) / 1e12,
+            "stage_ms": {**{k: round(v, 4) for k, v in st_p.items()},
+                         **{k: round(v, 4) for k, v in st_d.items()}},
+            "roofline": roofline,
+            "roofline_stages": stages,
+            "clocks": clk,
+            "gpu_launches": launches,
+            "e2e": {"value": world * K * pflops / (e2e_ms * 1e-3) / 1e12,
+                    "unit": "TFLOP/s", "h2d_bytes_per_step": x.numel() * 2,
+                    "d2h_bytes_per_step": out.numel() * 2,
+                    "what": "prefill through mla_prefill_forward with pinned host "
+                            "input/output copies inside the timed region"},
+            "source_hash": source_hash(),
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,110 @@
+// Internal declarations shared by the host API and the kernel launchers.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// Device status word bits (first 4 bytes of every workspace).
+enum : uint32_t {
+  kStatusTimeout = 1u << 0,   // a bounded wait ran out
+  kStatusBadCtx = 1u << 1,    // decode: a cu_ctx length outside [1, max_ctx]
+};
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float load(const float* p) { return *p; }
+  static __device__ __forceinline__ void store(float* p, float v) { *p = v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float v) {
+    *p = __float2bfloat16_rn(v);
+  }
+};
+
+// One column segment of a GEMM output and the epilogue applied to it.
+// Order of operations on an fp32 accumulator value v of row m, local col n:
+//   ssq_out[m] += v^2               for n < norm_cols           (pre-gain)
+//   v *= rsqrt(ssq_in[m] * rs_inv_dim + eps)        if ssq_in   (RMS scale)
+//   RoPE on cols with (n % rope_period) in [rope_start, rope_start+rope_dim)
+//        position = m % T, pairs (i, i + rope_dim/2)            if cos
+//   v *= gamma[n]                   for n < norm_cols           if gamma
+//   out[m * ldo + n] = v (rounded to the element type)
+struct EpiSeg {
+  void* out = nullptr;
+  int64_t ldo = 0;
+  int ncols = 0;
+  const void* gamma = nullptr;
+  int norm_cols = 0;
+  float* ssq_out = nullptr;
+  const float* ssq_in = nullptr;
+  float rs_inv_dim = 0.f;
+  float eps = 0.f;
+  const float* cos = nullptr;
+  const float* sin = nullptr;
+  int rope_period = 0, rope_start = 0, rope_dim = 0, T = 1;
+};
+
+// C = A B^T with A [M, K] (row stride lda) and the output columns split in up
+// to two segments: columns of segment s come from rows of Bs [ncols_s, K].
+struct GemmArgs {
+  const void* A = nullptr;
+  int64_t lda = 0;
+  const void* Bm[2] = {nullptr, nullptr};
+  int64_t ldb[2] = {0, 0};
+  int M = 0, K = 0;
+  int nseg = 1;
+  EpiSeg seg[2];
+};
+
+struct AttnArgs {
+  const void* q;        // [N, h, dq]
+  const void* kv;       // [N, h, dn+dv]
+  const void* ckv;      // [N, r_kv+dr]  (k_pe at column r_kv)
+  void* o;              // [N, h, dv]
+  int B, T, h, dn, dr, dv, r_kv;
+  float scale;
+  uint32_t* status;
+};
+
+struct DecodeArgs {
+  const void* q_nope;   // [B, h, dn]
+  const void* q_pe;     // [B, h, dr]
+  const void* w_kv_b;   // [h*(dn+dv), r]
+  const void* cache;    // [sum ctx, r + dr]
+  const int32_t* cu_ctx;
+  int B, max_ctx, h, dn, dr, dv, r;
+  float scale;
+  int split_tokens, max_splits;
+  void* q_lat;          // [B, h, r + dr]
+  float* part_o;        // [B, max_splits, h, r]
+  float* part_lse;      // [B, max_splits, h]
+  void* o_lat;          // [B, h, r]
+  void* o;              // [B, h, dv]
+  uint32_t* status;
+};
+
+// Launch accounting and stage events (defined in api.cu).
+void count_launches(int n = 1);
+// Records registered stage event i (if any) on stream st.
+void stage_event(int i, cudaStream_t st);
+
+// Launchers (return the launch error).
+cudaError_t launch_rope_tables(const mla_config& cfg, int max_pos, float* cos,
+                               float* sin, cudaStream_t st);
+cudaError_t launch_gemm_simt(int dtype, const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_attn_simt(int dtype, const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_latent_finalize(int dtype, const void* ckv,
+                                   const float* ssq_kv, int N, int r_kv,
+                                   int dr, float eps, void* cache,
+                                   cudaStream_t st);
+cudaError_t launch_decode_simt(int dtype, const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace mla

@@ -1,0 +1,16 @@
+// Tensor-core (tcgen05 / TMEM / TMA) path for sm_100a, bf16 operands.
+#pragma once
+#include "internal.h"
+
+namespace mla {
+
+// Whether the bf16 tensor-core kernels take this prefill configuration.
+bool tc_prefill_supported(const mla_config& c);
+// Whether a single GEMM can run on the tensor-core kernel.
+bool tc_gemm_supported(const GemmArgs& a, int dtype);
+cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status);
+cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st);
+bool tc_decode_supported(const mla_config& c);
+cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace mla

@@ -1,0 +1,56 @@
+"""Shared pieces of the GPU parity tests: run the C ABI on seeded inputs and
+bring results back as float64 numpy arrays."""
+import numpy as np
+import torch
+
+from latent_attention_b200.layer import MlaPrefill, MlaDecode
+
+# Tolerances on max|gpu - oracle| / max|oracle| per output tensor: 1e-5 for
+# the fp32 configuration, 2e-2 for bf16 storage with fp32 accumulation.
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+
+
+def f64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def weights_of(inp):
+    return {k: getattr(inp, k) for k in
+            ("w_q_a", "g_q_a", "w_q_b", "w_q", "w_kv_a", "g_kv_a", "w_kv_b",
+             "w_o")}
+
+
+def run_prefill(cfg, inp, latent=True):
+    B, T = inp.B, inp.T
+    layer = MlaPrefill(cfg, weights_of(inp), B, T)
+    x = inp.x.cuda()
+    cache = (torch.empty(B * T, cfg.kv_lora_rank + cfg.qk_rope_head_dim,
+                         dtype=layer.dtype, device="cuda") if latent else None)
+    out = layer(x, latent_cache_out=cache)
+    torch.cuda.synchronize()
+    layer.check_status()
+    return layer, out, cache
+
+
+def sample_rows(T, n=64, seed=0):
+    g = np.random.default_rng(seed)
+    k = min(T, n)
+    edge = min(T, k // 4)
+    rows = set(range(edge)) | set(range(T - edge, T))
+    rest = [r for r in range(T) if r not in rows]
+    need = k - len(rows)
+    if need > 0 and rest:
+        rows |= set(g.choice(rest, size=min(need, len(rest)), replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+def run_decode(cfg, di, max_ctx, with_o=False):
+    B = di.q_nope.shape[0]
+    dec = MlaDecode(cfg, B, max_ctx)
+    H = cfg.hidden_size if with_o else cfg.num_heads * cfg.v_head_dim
+    out = torch.empty(B, H, dtype=dec.dtype, device="cuda")
+    dec(di.q_nope.cuda(), di.q_pe.cuda(), di.w_kv_b.cuda(), di.cache.cuda(),
+        di.cu_ctx.cuda(), out, di.w_o.cuda() if with_o else None)
+    torch.cuda.synchronize()
+    dec.check_status()
+    return dec, out

@@ -1,0 +1,169 @@
+"""GPU parity: the sm_100a library (through the C ABI) against the fp64 oracle
+on the same seeded inputs.  Small cases compare every output element; the
+full-size workloads compare sampled rows / sequences that the oracle computes
+one by one.  Tolerance: max|gpu - oracle| / max|oracle| <= 1e-5 (fp32) or
+2e-2 (bf16)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_inputs import (MlaConfig, WORKLOADS, make_prefill_inputs,
+                        make_decode_inputs, decode_context_lengths)
+from gpu_helpers import TOL, f64, run_prefill, run_decode, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+W = WORKLOADS
+
+
+def small_bf16(**kw):
+    """DeepSeek-V3 head dims at a small hidden size."""
+    base = dict(hidden_size=512, num_heads=4, q_lora_rank=256,
+                kv_lora_rank=512, qk_nope_head_dim=128, qk_rope_head_dim=64,
+                v_head_dim=128, rope_type="yarn", rope_theta=1e4,
+                rope_factor=40.0, rope_mscale=1.0, rope_mscale_all_dim=1.0,
+                original_max_position_embeddings=4096, dtype="bf16")
+    base.update(kw)
+    return MlaConfig(**base)
+
+
+# --------------------------------------------------------------------------
+# RoPE tables
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("name,max_pos", [("tiny_f32", 64), ("dsv3_prefill", 32768),
+                                          ("directq_prefill", 8192),
+                                          ("kimi_prefill", 16)])
+def test_rope_tables(cuda, name, max_pos):
+    from latent_attention_b200 import mla_build_rope_tables
+    cfg = W[name].cfg
+    d = cfg.qk_rope_head_dim
+    cos = torch.empty(max_pos, d, device=cuda)
+    sin = torch.empty_like(cos)
+    mla_build_rope_tables(cfg, max_pos, cos, sin)
+    torch.cuda.synchronize()
+    if cfg.rope_type == "none":
+        assert torch.all(cos == 1) and torch.all(sin == 0)
+        return
+    rc, rs = oracle.rope_tables(cfg, max_pos)
+    # one fp32 rounding of an fp64 value of magnitude <= 1
+    assert np.max(np.abs(f64(cos) - rc)) <= 1.2e-7
+    assert np.max(np.abs(f64(sin) - rs)) <= 1.2e-7
+
+
+# --------------------------------------------------------------------------
+# Prefill, every element, small shapes (several tiles + ragged tails)
+# --------------------------------------------------------------------------
+PREFILL_SMALL = [
+    ("tiny_f32", W["tiny_f32"].cfg, 1, 64, "ones"),
+    ("tiny_f32_b2_ragged_gamma", W["tiny_f32"].cfg, 2, 37, "random"),
+    ("tiny_f32_directq", W["tiny_f32"].cfg.with_(q_lora_rank=0), 1, 50, "ones"),
+    ("tiny_f32_norope", W["tiny_f32"].cfg.with_(rope_type="none"), 1, 33, "ones"),
+    ("tiny_f32_T1", W["tiny_f32"].cfg, 3, 1, "random"),
+    ("bf16_dsv3dims_ragged", small_bf16(), 2, 300, "random"),
+    ("bf16_directq", small_bf16(q_lora_rank=0, rope_type="plain", num_heads=2),
+     1, 257, "ones"),
+    ("bf16_kimi_norope", small_bf16(rope_type="none", num_heads=3), 1, 200, "ones"),
+    ("bf16_T1", small_bf16(), 2, 1, "ones"),
+]
+
+
+@pytest.mark.parametrize("name,cfg,B,T,gamma", PREFILL_SMALL,
+                         ids=[c[0] for c in PREFILL_SMALL])
+def test_prefill_small(cuda, name, cfg, B, T, gamma):
+    inp = make_prefill_inputs(cfg, B, T, seed=1, gamma=gamma)
+    layer, out, cache = run_prefill(cfg, inp)
+    ref, P = oracle.prefill(cfg, inp, return_parts=True)
+    tol = TOL[cfg.dtype]
+    assert oracle.max_rel_err(out, ref) <= tol
+    # the latent cache handed to decode: [RMSNorm(c) | roped k_pe]
+    assert oracle.max_rel_err(cache.view(B, T, -1), P["latent_cache"]) <= tol
+    # intermediates: roped queries and the per-head k_nope | V
+    N, h = B * T, cfg.num_heads
+    dq = cfg.qk_head_dim
+    q = f64(layer.view("q", (B, T, h, dq)))
+    assert oracle.max_rel_err(q[..., :cfg.qk_nope_head_dim], P["q_nope"]) <= tol
+    assert oracle.max_rel_err(q[..., cfg.qk_nope_head_dim:], P["q_pe"]) <= tol
+    kv = f64(layer.view("kv", (B, T, h, cfg.qk_nope_head_dim + cfg.v_head_dim)))
+    assert oracle.max_rel_err(kv[..., :cfg.qk_nope_head_dim], P["k_nope"]) <= tol
+    assert oracle.max_rel_err(kv[..., cfg.qk_nope_head_dim:], P["v"]) <= tol
+    attn = f64(layer.view("attn", (B, T, h, cfg.v_head_dim)))
+    assert oracle.max_rel_err(attn, P["attn"]) <= tol
+
+
+def test_prefill_is_deterministic_and_overwrites(cuda):
+    cfg = small_bf16()
+    inp = make_prefill_inputs(cfg, 1, 130, seed=2)
+    layer, out1, _ = run_prefill(cfg, inp)
+    first = out1.clone()
+    out1.fill_(float("nan"))
+    layer(inp.x.cuda(), out=out1)
+    torch.cuda.synchronize()
+    assert torch.equal(first, out1)
+
+
+# --------------------------------------------------------------------------
+# Prefill at the full workload sizes: sampled rows
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["dsv3_prefill", "directq_prefill", "kimi_prefill"])
+def test_prefill_full_size_sampled_rows(cuda, name):
+    wl = W[name]
+    cfg = wl.cfg
+    inp = make_prefill_inputs(cfg, wl.batch, wl.seq_len, seed=0)
+    layer, out, _ = run_prefill(cfg, inp, latent=False)
+    rows = sample_rows(wl.seq_len, 48)
+    bsel = [0, wl.batch - 1] if wl.batch > 1 else [0]
+    sub = type(inp)(**{**inp.__dict__, "x": inp.x[bsel], "B": len(bsel)})
+    ref = oracle.prefill(cfg, sub, rows=rows)
+    got = out[bsel][:, torch.as_tensor(rows)]
+    assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
+
+
+# --------------------------------------------------------------------------
+# Absorbed decode
+# --------------------------------------------------------------------------
+DECODE_SMALL = [
+    ("tiny_f32", W["tiny_f32"].cfg, [1, 7, 64, 130], 200),
+    ("bf16_dsv3dims", small_bf16(), [1, 5, 300, 2049, 77], 4096),
+    ("bf16_dsv3_heads", W["dsv3_decode"].cfg, [1, 1000, 33], 1024),
+]
+
+
+@pytest.mark.parametrize("name,cfg,ctx,max_ctx", DECODE_SMALL,
+                         ids=[c[0] for c in DECODE_SMALL])
+@pytest.mark.parametrize("with_o", [False, True])
+def test_decode_small(cuda, name, cfg, ctx, max_ctx, with_o):
+    B = len(ctx)
+    di = make_decode_inputs(cfg, B, ctx, seed=3, with_o_proj=with_o)
+    _, out = run_decode(cfg, di, max_ctx, with_o)
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache,
+                                 di.cu_ctx, di.w_o if with_o else None)
+    assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
+
+
+def test_decode_full_size_sampled_sequences(cuda):
+    wl = W["dsv3_decode"]
+    cfg = wl.cfg
+    ctx = decode_context_lengths(wl.batch, wl.ctx_min, wl.ctx_max, seed=0)
+    di = make_decode_inputs(cfg, wl.batch, ctx, seed=0)
+    _, out = run_decode(cfg, di, wl.ctx_max)
+    order = np.argsort(ctx.numpy())
+    picks = sorted({int(order[0]), int(order[-1]), 17})
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache,
+                                 di.cu_ctx, batches=picks)
+    assert oracle.max_rel_err(out[picks], ref) <= TOL[cfg.dtype]
+
+
+def test_decode_bad_context_is_flagged(cuda):
+    from latent_attention_b200 import MlaError
+    cfg = small_bf16()
+    di = make_decode_inputs(cfg, 2, [5, 9], seed=4)
+    from latent_attention_b200.layer import MlaDecode
+    dec = MlaDecode(cfg, 2, 8)               # max_ctx 8 < 9
+    out = torch.empty(2, cfg.num_heads * cfg.v_head_dim, dtype=torch.bfloat16,
+                      device=cuda)
+    dec(di.q_nope.cuda(), di.q_pe.cuda(), di.w_kv_b.cuda(), di.cache.cuda(),
+        di.cu_ctx.cuda(), out)
+    with pytest.raises(MlaError, match="MLA_ERR_SHAPE"):
+        dec.check_status()
+    dec.check_status()                       # the word was cleared
