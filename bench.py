@@ -305,6 +305,12 @@ def main():
     ev_p = [[mk() for _ in range(6)] for _ in range(K)]
     ev_d = [[mk() for _ in range(6)] for _ in range(K)]
     ev_s = [(mk(), mk()) for _ in range(K)]
+    # torch creates the CUDA event lazily at its first record; the library
+    # records through the raw handle, so materialise every handle now.
+    for group in ev_p + ev_d:
+        for e in group:
+            e.record()
+    torch.cuda.synchronize()
 
     def set_events(evs):
         if evs is None:

@@ -101,8 +101,10 @@ void prefill_layout(const mla_config& c, int B, int T, mla_prefill_layout* L) {
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off = align256(off + bytes); return o; };
   L->status = take(256);
-  L->ssq_q = c.q_lora_rank > 0 ? take(N * 4) : -1;
-  L->ssq_kv = take(N * 4);
+  // RMS statistics: one partial sum per 64-column tile (the narrowest
+  // producer tile) and row.
+  L->ssq_q = c.q_lora_rank > 0 ? take(N * 4 * ((c.q_lora_rank + 63) / 64)) : -1;
+  L->ssq_kv = take(N * 4 * ((c.kv_lora_rank + 63) / 64));
   L->q_a = c.q_lora_rank > 0 ? take(N * c.q_lora_rank * es) : -1;
   L->ckv = take(N * (c.kv_lora_rank + c.qk_rope_head_dim) * es);
   L->q = take(N * c.num_heads * dq * es);
@@ -227,14 +229,13 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
   const int h = c.num_heads, dn = c.qk_nope_head_dim, dr = c.qk_rope_head_dim, dv = c.v_head_dim;
   const int dq = dn + dr, r_kv = c.kv_lora_rank, H = c.hidden_size;
   const float eps = (float)c.rms_eps;
-  const bool tc = mla::tc_prefill_supported(c);
-  if (!tc) {
-    if (rope && (!rope_fits_simt_tiles(dq, dn, dr, h) ||
-                 !rope_fits_simt_tiles(r_kv + dr, r_kv, dr, 1)))
-      return fail(MLA_ERR_UNSUPPORTED, "rope columns straddle a 64-column tile");
-    if (sizeof(float) * (16 * dq + 32 * dq + 32 * dv + 16 * 32 + 16 * dv + 48) > 227 * 1024)
-      return fail(MLA_ERR_UNSUPPORTED, "head dims too large for the CUDA-core attention");
-  }
+  const bool tc_attn = mla::tc_attention_supported(c);
+  if (rope && (!rope_fits_simt_tiles(dq, dn, dr, h) ||
+               !rope_fits_simt_tiles(r_kv + dr, r_kv, dr, 1)) && c.dtype == MLA_F32)
+    return fail(MLA_ERR_UNSUPPORTED, "rope columns straddle a 64-column tile");
+  if (!tc_attn &&
+      sizeof(float) * (16 * dq + 32 * dq + 32 * dv + 16 * 32 + 16 * dv + 48) > 227 * 1024)
+    return fail(MLA_ERR_UNSUPPORTED, "head dims too large for the CUDA-core attention");
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = static_cast<char*>(workspace);
   float* ssq_q = (float*)at(ws, L.ssq_q);
@@ -246,9 +247,8 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
   void* attn = at(ws, L.attn);
   uint32_t* status = (uint32_t*)at(ws, L.status);
 
-  // status word + RMS row statistics start at zero (they are contiguous).
-  const int64_t zero_end = L.q_a >= 0 ? L.q_a : L.ckv;
-  cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)zero_end, st);
+  // The status word starts at zero; every other buffer is fully written.
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   mla::stage_event(0, st);
 
@@ -261,14 +261,14 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
     mla::EpiSeg& e0 = g.seg[si];
     g.Bm[si] = w->w_q_a; g.ldb[si] = H;
     e0.out = q_a; e0.ldo = c.q_lora_rank; e0.ncols = c.q_lora_rank;
-    e0.gamma = w->g_q_a; e0.norm_cols = c.q_lora_rank; e0.ssq_out = ssq_q;
+    e0.gamma = w->g_q_a; e0.norm_cols = c.q_lora_rank; e0.ssq_out = ssq_q; e0.ssq_ld = N;
     ++si;
   }
   {
     mla::EpiSeg& e1 = g.seg[si];
     g.Bm[si] = w->w_kv_a; g.ldb[si] = H;
     e1.out = ckv; e1.ldo = r_kv + dr; e1.ncols = r_kv + dr;
-    e1.gamma = w->g_kv_a; e1.norm_cols = r_kv; e1.ssq_out = ssq_kv;
+    e1.gamma = w->g_kv_a; e1.norm_cols = r_kv; e1.ssq_out = ssq_kv; e1.ssq_ld = N;
     if (rope) {
       e1.cos = rope_cos; e1.sin = rope_sin; e1.rope_period = r_kv + dr;
       e1.rope_start = r_kv; e1.rope_dim = dr; e1.T = T;
@@ -276,7 +276,18 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
     ++si;
   }
   g.nseg = si;
-  e = tc ? mla::tc_gemm(g, st, status) : mla::launch_gemm_simt(c.dtype, g, st);
+  // Each projection runs on the tensor-core GEMM when it takes the shape;
+  // the column tile of the down-projection fixes the RMS partial count.
+  auto run_gemm = [&](const mla::GemmArgs& ga) {
+    if (mla::tc_gemm_supported(ga, c.dtype)) return mla::tc_gemm(ga, st, status);
+    if (ga.seg[0].cos && !rope_fits_simt_tiles(ga.seg[0].rope_period, ga.seg[0].rope_start,
+                                               ga.seg[0].rope_dim,
+                                               ga.seg[0].ncols / ga.seg[0].rope_period))
+      return cudaErrorNotSupported;
+    return mla::launch_gemm_simt(c.dtype, ga, st);
+  };
+  const int tile_n = mla::tc_gemm_supported(g, c.dtype) ? mla::kTcTileN : mla::kSimtTileN;
+  e = run_gemm(g);
   if (e != cudaSuccess) return cuda_fail(e, "down-projection");
   mla::stage_event(1, st);
 
@@ -288,6 +299,7 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
     gq.A = q_a; gq.lda = c.q_lora_rank; gq.K = c.q_lora_rank;
     gq.Bm[0] = w->w_q_b; gq.ldb[0] = c.q_lora_rank;
     eq.ssq_in = ssq_q; eq.rs_inv_dim = 1.0f / c.q_lora_rank; eq.eps = eps;
+    eq.ssq_parts = (c.q_lora_rank + tile_n - 1) / tile_n; eq.ssq_ld = N;
   } else {
     gq.A = x; gq.lda = H; gq.K = H;
     gq.Bm[0] = w->w_q; gq.ldb[0] = H;
@@ -297,7 +309,7 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
     eq.cos = rope_cos; eq.sin = rope_sin; eq.rope_period = dq; eq.rope_start = dn;
     eq.rope_dim = dr; eq.T = T;
   }
-  e = tc ? mla::tc_gemm(gq, st, status) : mla::launch_gemm_simt(c.dtype, gq, st);
+  e = run_gemm(gq);
   if (e != cudaSuccess) return cuda_fail(e, "q projection");
   mla::stage_event(2, st);
 
@@ -308,13 +320,14 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
   mla::EpiSeg& ek = gk.seg[0];
   ek.out = kv; ek.ldo = (int64_t)h * (dn + dv); ek.ncols = h * (dn + dv);
   ek.ssq_in = ssq_kv; ek.rs_inv_dim = 1.0f / r_kv; ek.eps = eps;
-  e = tc ? mla::tc_gemm(gk, st, status) : mla::launch_gemm_simt(c.dtype, gk, st);
+  ek.ssq_parts = (r_kv + tile_n - 1) / tile_n; ek.ssq_ld = N;
+  e = run_gemm(gk);
   if (e != cudaSuccess) return cuda_fail(e, "kv up-projection");
   mla::stage_event(3, st);
 
   // S7: causal attention.
   mla::AttnArgs aa{q, kv, ckv, attn, B, T, h, dn, dr, dv, r_kv, (float)softmax_scale(c), status};
-  e = tc ? mla::tc_attention(aa, st) : mla::launch_attn_simt(c.dtype, aa, st);
+  e = tc_attn ? mla::tc_attention(aa, st) : mla::launch_attn_simt(c.dtype, aa, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   mla::stage_event(4, st);
 
@@ -323,12 +336,13 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
   go.A = attn; go.lda = (int64_t)h * dv; go.M = N; go.K = h * dv; go.nseg = 1;
   go.Bm[0] = w->w_o; go.ldb[0] = (int64_t)h * dv;
   go.seg[0].out = out; go.seg[0].ldo = H; go.seg[0].ncols = H;
-  e = tc ? mla::tc_gemm(go, st, status) : mla::launch_gemm_simt(c.dtype, go, st);
+  e = run_gemm(go);
   if (e != cudaSuccess) return cuda_fail(e, "o_proj");
   mla::stage_event(5, st);
 
   if (latent_cache_out) {
-    e = mla::launch_latent_finalize(c.dtype, ckv, ssq_kv, N, r_kv, dr, eps, latent_cache_out, st);
+    e = mla::launch_latent_finalize(c.dtype, ckv, ssq_kv, (r_kv + tile_n - 1) / tile_n, N, r_kv,
+                                    dr, eps, latent_cache_out, st);
     if (e != cudaSuccess) return cuda_fail(e, "latent cache");
   }
   g_detail.clear();

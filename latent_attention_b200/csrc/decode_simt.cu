@@ -18,7 +18,7 @@ namespace {
 
 template <typename T>
 __global__ void latent_finalize_kernel(const T* __restrict__ ckv,
-                                       const float* __restrict__ ssq, int N,
+                                       const float* __restrict__ ssq, int parts, int N,
                                        int r, int dr, float eps,
                                        T* __restrict__ cache) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -27,7 +27,11 @@ __global__ void latent_finalize_kernel(const T* __restrict__ ckv,
   const int64_t m = idx / w;
   const int c = (int)(idx % w);
   float v = Elem<T>::load(ckv + idx);
-  if (c < r) v *= rsqrtf(ssq[m] * (1.0f / r) + eps);
+  if (c < r) {
+    float ss = 0.f;
+    for (int p = 0; p < parts; ++p) ss += ssq[(int64_t)p * N + m];
+    v *= rsqrtf(ss * (1.0f / r) + eps);
+  }
   Elem<T>::store(cache + idx, v);
 }
 
@@ -182,17 +186,17 @@ cudaError_t run_decode(const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_latent_finalize(int dtype, const void* ckv, const float* ssq_kv,
-                                   int N, int r_kv, int dr, float eps, void* cache,
+                                   int ssq_parts, int N, int r_kv, int dr, float eps, void* cache,
                                    cudaStream_t st) {
   const int64_t total = (int64_t)N * (r_kv + dr);
   const unsigned blocks = (unsigned)((total + 255) / 256);
   count_launches();
   if (dtype == MLA_F32)
     latent_finalize_kernel<float><<<blocks, 256, 0, st>>>(
-        (const float*)ckv, ssq_kv, N, r_kv, dr, eps, (float*)cache);
+        (const float*)ckv, ssq_kv, ssq_parts, N, r_kv, dr, eps, (float*)cache);
   else
     latent_finalize_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)ckv, ssq_kv, N, r_kv, dr, eps, (__nv_bfloat16*)cache);
+        (const __nv_bfloat16*)ckv, ssq_kv, ssq_parts, N, r_kv, dr, eps, (__nv_bfloat16*)cache);
   return cudaGetLastError();
 }
 

@@ -11,7 +11,7 @@
 namespace mla {
 namespace {
 
-constexpr int BM = 64, BN = 64, BK = 16, NT = 256;
+constexpr int BM = 64, BN = kSimtTileN, BK = 16, NT = 256;
 
 template <typename T>
 __device__ __forceinline__ float ld(const void* p, int64_t i) {
@@ -75,7 +75,11 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(GemmArgs a) {
   const int m = m0 + r;
   if (m >= a.M) return;
   float rs = 1.f;
-  if (e.ssq_in) rs = rsqrtf(e.ssq_in[m] * e.rs_inv_dim + e.eps);
+  if (e.ssq_in) {
+    float ss = 0.f;
+    for (int p = 0; p < e.ssq_parts; ++p) ss += e.ssq_in[p * e.ssq_ld + m];
+    rs = rsqrtf(ss * e.rs_inv_dim + e.eps);
+  }
   float ssq = 0.f;
   const int pos = m % e.T;
   T* out = reinterpret_cast<T*>(e.out);
@@ -102,7 +106,7 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(GemmArgs a) {
   if (e.ssq_out) {
     ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
     ssq += __shfl_xor_sync(0xffffffffu, ssq, 2);
-    if ((tid % 4) == 0 && n0 < e.norm_cols) atomicAdd(e.ssq_out + m, ssq);
+    if ((tid % 4) == 0 && n0 < e.norm_cols) e.ssq_out[tile_n * e.ssq_ld + m] = ssq;
   }
 }
 

@@ -1,0 +1,315 @@
+// tcgen05 GEMM for the MLA projections (bf16 in, fp32 TMEM accumulators).
+//
+// C = A B^T, A [M, K] and B [N, K] both K-major (nn.Linear [out, in] weights,
+// MiniMind "Attention 前向传播" section 2), output columns split in up to two
+// segments with their own B matrix (the fused q_a | kv_a down-projection of
+// the CSDN DeepseekV3Attention forward shares the input x).
+//
+// Persistent, warp-specialised kernel, one CTA per SM:
+//   warp 0      TMA producer: 128x64 A box + 256x64 B box per stage,
+//               128-byte swizzle, 4-stage ring of mbarriers
+//   warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma M128 N256 K16
+//               per stage into one of two TMEM accumulators (2 x 256 columns)
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = row), the
+//               fused RMSNorm statistics / row scale / gain and RoPE of the
+//               rope columns (see EpiSeg), bf16 stores.
+// The two TMEM accumulators let the epilogue of tile i overlap the MMAs of
+// tile i+1.  Every mbarrier wait is bounded (sm100::mbar_wait).
+#include "sm100.cuh"
+#include "tc.h"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = kTcTileN, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr int NTHREADS = 192;
+constexpr uint32_t IDESC = idesc_bf16(BM, BN);
+constexpr uint32_t TMEM_COLS = 2 * BN;
+
+struct TcGemmParams {
+  int M, K;
+  int nseg;
+  int tiles_m;
+  int tiles_n[2];
+  int total_tiles;
+  EpiSeg seg[2];
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& s, int& m0,
+                                            int& n0) {
+  const int first = p.tiles_m * p.tiles_n[0];
+  s = (t >= first) ? 1 : 0;
+  const int local = s ? t - first : t;
+  m0 = (local % p.tiles_m) * BM;
+  n0 = (local / p.tiles_m) * BN;
+}
+
+// Epilogue of one 128 x BN tile; this thread owns output row m0 + row.
+__device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSeg& e, int m0,
+                                              int n0, int row, uint32_t taddr) {
+  const int m = m0 + row;
+  const bool row_ok = m < p.M;
+  float rs = 1.f;
+  if (e.ssq_in && row_ok) {
+    float ss = 0.f;
+    for (int q = 0; q < e.ssq_parts; ++q) ss += e.ssq_in[q * e.ssq_ld + m];
+    rs = rsqrtf(ss * e.rs_inv_dim + e.eps);
+  }
+  const int pos = row_ok ? m % e.T : 0;
+  float ssq = 0.f;
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out);
+  const __nv_bfloat16* gamma = reinterpret_cast<const __nv_bfloat16*>(e.gamma);
+#pragma unroll 1
+  for (int g = 0; g < BN / 64; ++g) {
+    const int nl = n0 + g * 64;
+    if (nl >= e.ncols) break;  // uniform over the warp
+    uint32_t r0[32], r1[32];
+    tmem_ld32(taddr + g * 64, r0);
+    tmem_ld32(taddr + g * 64 + 32, r1);
+    tmem_wait_ld();
+    float v[64];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      v[i] = __uint_as_float(r0[i]);
+      v[i + 32] = __uint_as_float(r1[i]);
+    }
+    if (e.ssq_out) {
+      const int lim = e.norm_cols - nl;
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (i < lim) ssq = fmaf(v[i], v[i], ssq);
+    }
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] *= rs;
+    if (e.cos && (nl % e.rope_period) == e.rope_start) {
+      // rotate_half RoPE on a 64-wide rope segment: pairs (i, i + 32).
+      const float4* cs = reinterpret_cast<const float4*>(e.cos + (int64_t)pos * 64);
+      const float4* sn = reinterpret_cast<const float4*>(e.sin + (int64_t)pos * 64);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 c1 = __ldg(cs + j), s1 = __ldg(sn + j);
+        const float4 c2 = __ldg(cs + j + 8), s2 = __ldg(sn + j + 8);
+        const float cc1[4] = {c1.x, c1.y, c1.z, c1.w}, ss1[4] = {s1.x, s1.y, s1.z, s1.w};
+        const float cc2[4] = {c2.x, c2.y, c2.z, c2.w}, ss2[4] = {s2.x, s2.y, s2.z, s2.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = 4 * j + k;
+          const float x1 = v[i], x2 = v[i + 32];
+          v[i] = x1 * cc1[k] - x2 * ss1[k];
+          v[i + 32] = x2 * cc2[k] + x1 * ss2[k];
+        }
+      }
+    }
+    if (gamma && nl < e.norm_cols) {
+      const int lim = e.norm_cols - nl;
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (i < lim) v[i] *= __bfloat162float(gamma[nl + i]);
+    }
+    if (row_ok) {
+      __nv_bfloat16* dst = out + (int64_t)m * e.ldo + nl;
+      const int lim = e.ncols - nl;
+#pragma unroll
+      for (int c = 0; c < 64; c += 8) {
+        if (c < lim)
+          st_global_v4(dst + c, pack_bf16(v[c], v[c + 1]), pack_bf16(v[c + 2], v[c + 3]),
+                       pack_bf16(v[c + 4], v[c + 5]), pack_bf16(v[c + 6], v[c + 7]));
+      }
+    }
+  }
+  if (e.ssq_out && row_ok && n0 < e.norm_cols) e.ssq_out[(n0 / BN) * e.ssq_ld + m] = ssq;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ TcGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2];
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  volatile int* abort_v = &abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB0);
+    if (p.nseg > 1) tma_prefetch(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base, TMEM_COLS);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+  const int nk = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+        int s, m0, n0;
+        tile_coords(p, t, s, m0, n0);
+        const CUtensorMap* tmB = s ? &tmB1 : &tmB0;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_v, p.status)) goto done;
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sa, &tmA, kb * BK, m0, &full[stage]);
+          tma_load_2d(sa + A_BYTES, tmB, kb * BK, n0, &full[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t tph = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], tph ^ 1, abort_v, p.status)) goto done;
+        tc_fence_after();
+        const uint32_t d = tbase + buf * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_v, p.status)) goto done;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), IDESC,
+                     (kb | k) != 0);
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        mma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
+      const int buf = local & 1;
+      const uint32_t tph = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[buf], tph, abort_v, p.status)) break;
+      tc_fence_after();
+      int s, m0, n0;
+      tile_coords(p, t, s, m0, n0);
+      epilogue_tile(p, p.seg[s], m0, n0, row, tbase + ((uint32_t)(quad * 32) << 16) + buf * BN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+done:
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool tc_gemm_supported(const GemmArgs& a, int dtype) {
+  if (dtype != MLA_BF16 || a.M < 1 || a.K < 1) return false;
+  if (a.K % 8 || a.lda % 8 || !aligned16(a.A)) return false;
+  for (int s = 0; s < a.nseg; ++s) {
+    const EpiSeg& e = a.seg[s];
+    if (a.ldb[s] % 8 || !aligned16(a.Bm[s]) || !aligned16(e.out)) return false;
+    if (e.ncols < 1 || e.ncols % 8 || e.ldo % 8) return false;
+    if (e.cos && (e.rope_dim != 64 || e.rope_start % 64 || e.rope_period % 64)) return false;
+    if (e.ssq_in && e.ssq_parts < 1) return false;
+  }
+  return true;
+}
+
+cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
+  CUtensorMap tmA, tmB[2];
+  {
+    const uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
+    const uint64_t strides[1] = {(uint64_t)a.lda * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!encode_tmap(&tmA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  TcGemmParams p{};
+  p.M = a.M;
+  p.K = a.K;
+  p.nseg = a.nseg;
+  p.tiles_m = (a.M + BM - 1) / BM;
+  p.total_tiles = 0;
+  for (int s = 0; s < a.nseg; ++s) {
+    const uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.seg[s].ncols};
+    const uint64_t strides[1] = {(uint64_t)a.ldb[s] * 2};
+    const uint32_t box[2] = {BK, BN};
+    if (!encode_tmap(&tmB[s], a.Bm[s], 2, dims, strides, box)) return cudaErrorInvalidValue;
+    p.seg[s] = a.seg[s];
+    p.tiles_n[s] = (a.seg[s].ncols + BN - 1) / BN;
+    p.total_tiles += p.tiles_m * p.tiles_n[s];
+  }
+  if (a.nseg == 1) {
+    tmB[1] = tmB[0];
+    p.tiles_n[1] = 0;
+  }
+  p.status = status;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
+  gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmA, tmB[0], tmB[1], p);
+  count_launches();
+  return cudaGetLastError();
+}
+
+}  // namespace mla

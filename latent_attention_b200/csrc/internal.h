@@ -31,8 +31,10 @@ template <> struct Elem<__nv_bfloat16> {
 
 // One column segment of a GEMM output and the epilogue applied to it.
 // Order of operations on an fp32 accumulator value v of row m, local col n:
-//   ssq_out[m] += v^2               for n < norm_cols           (pre-gain)
-//   v *= rsqrt(ssq_in[m] * rs_inv_dim + eps)        if ssq_in   (RMS scale)
+//   ssq_out[tile * ssq_ld + m] = sum v^2 over the tile's cols < norm_cols
+//                                   (pre-gain partial, one per column tile)
+//   v *= rsqrt(sum_p ssq_in[p * ssq_ld + m] * rs_inv_dim + eps)   if ssq_in
+//                                   (RMS row scale; partials summed in order)
 //   RoPE on cols with (n % rope_period) in [rope_start, rope_start+rope_dim)
 //        position = m % T, pairs (i, i + rope_dim/2)            if cos
 //   v *= gamma[n]                   for n < norm_cols           if gamma
@@ -45,6 +47,8 @@ struct EpiSeg {
   int norm_cols = 0;
   float* ssq_out = nullptr;
   const float* ssq_in = nullptr;
+  int ssq_parts = 0;        // partial count to sum for ssq_in
+  int64_t ssq_ld = 0;       // row count of the partial buffer (M)
   float rs_inv_dim = 0.f;
   float eps = 0.f;
   const float* cos = nullptr;
@@ -100,9 +104,11 @@ void stage_event(int i, cudaStream_t st);
 cudaError_t launch_rope_tables(const mla_config& cfg, int max_pos, float* cos,
                                float* sin, cudaStream_t st);
 cudaError_t launch_gemm_simt(int dtype, const GemmArgs& a, cudaStream_t st);
+// Column tile width of the CUDA-core GEMM (RMS partial count = ceil(cols/64)).
+constexpr int kSimtTileN = 64;
 cudaError_t launch_attn_simt(int dtype, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_latent_finalize(int dtype, const void* ckv,
-                                   const float* ssq_kv, int N, int r_kv,
+                                   const float* ssq_kv, int ssq_parts, int N, int r_kv,
                                    int dr, float eps, void* cache,
                                    cudaStream_t st);
 cudaError_t launch_decode_simt(int dtype, const DecodeArgs& a, cudaStream_t st);

@@ -4,8 +4,11 @@
 
 namespace mla {
 
-// Whether the bf16 tensor-core kernels take this prefill configuration.
-bool tc_prefill_supported(const mla_config& c);
+// Column tile width of the tensor-core GEMM.
+constexpr int kTcTileN = 256;
+
+// Whether the tensor-core attention kernel takes this configuration.
+bool tc_attention_supported(const mla_config& c);
 // Whether a single GEMM can run on the tensor-core kernel.
 bool tc_gemm_supported(const GemmArgs& a, int dtype);
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status);
