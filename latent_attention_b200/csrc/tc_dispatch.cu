@@ -3,8 +3,6 @@
 
 namespace mla {
 
-bool tc_attention_supported(const mla_config&) { return false; }
-cudaError_t tc_attention(const AttnArgs&, cudaStream_t) { return cudaErrorNotSupported; }
 bool tc_decode_supported(const mla_config&) { return false; }
 cudaError_t tc_decode(const DecodeArgs&, cudaStream_t) { return cudaErrorNotSupported; }
 

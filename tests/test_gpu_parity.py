@@ -91,6 +91,25 @@ def test_prefill_small(cuda, name, cfg, B, T, gamma):
     assert oracle.max_rel_err(attn, P["attn"]) <= tol
 
 
+@pytest.mark.parametrize("profile", ["growing", "shrinking", "large"])
+def test_prefill_softmax_range_stress(cuda, profile):
+    """Inputs whose attention scores grow (or shrink) along the sequence, so
+    that the running row maximum keeps increasing and the kernels must rescale
+    their partial outputs, plus a case with a large score range."""
+    cfg = small_bf16(q_lora_rank=0, rope_type="plain", num_heads=2)
+    T = 520
+    inp = make_prefill_inputs(cfg, 1, T, seed=5)
+    t = torch.arange(T, dtype=torch.float32)
+    f = {"growing": 1 + 6 * t / T, "shrinking": 7 - 6 * t / T,
+         "large": torch.full((T,), 6.0)}[profile]
+    inp.x = (inp.x.float() * f[None, :, None]).to(torch.bfloat16)
+    layer, out, cache = run_prefill(cfg, inp)
+    ref, P = oracle.prefill(cfg, inp, return_parts=True)
+    attn = f64(layer.view("attn", (1, T, cfg.num_heads, cfg.v_head_dim)))
+    assert oracle.max_rel_err(attn, P["attn"]) <= TOL["bf16"]
+    assert oracle.max_rel_err(out, ref) <= TOL["bf16"]
+
+
 def test_prefill_is_deterministic_and_overwrites(cuda):
     cfg = small_bf16()
     inp = make_prefill_inputs(cfg, 1, 130, seed=2)
