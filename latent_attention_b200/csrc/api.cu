@@ -113,7 +113,9 @@ void prefill_layout(const mla_config& c, int B, int T, mla_prefill_layout* L) {
   L->total_bytes = off;
 }
 
-int decode_split_tokens(const mla_config& c) { (void)c; return 1024; }
+int decode_split_tokens(const mla_config& c) {
+  return mla::tc_decode_supported(c) ? mla::tc_decode_split_tokens() : 1024;
+}
 
 void decode_layout(const mla_config& c, int B, int max_ctx, mla_decode_layout* L) {
   const int64_t es = elem_size(c);
@@ -379,6 +381,8 @@ mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope, const 
   if ((int64_t)workspace_bytes < L.total_bytes)
     return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
                 (long long)L.total_bytes);
+  if (mla::tc_decode_supported(c) && L.max_splits > 64)
+    return fail(MLA_ERR_UNSUPPORTED, "max_ctx=%d needs more than 64 splits", max_ctx);
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);

@@ -54,19 +54,6 @@ struct AttnTcParams {
   uint32_t* status;
 };
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmKV,
@@ -198,7 +185,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const int slot = j & 1;
-      if (!mbar_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
+      if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
@@ -224,7 +211,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int i = 0; i < 128; ++i) mx = fmaxf(mx, s[i]);
       const bool grow = mx > m_ref + kRescaleLog2;    // also true for the first block
       if (j > 0) {
-        if (!mbar_wait(&pv_done, (j - 1) & 1, abort_v, p.status)) { ok = false; break; }
+        if (!warp_wait(&pv_done, (j - 1) & 1, abort_v, p.status)) { ok = false; break; }
         tc_fence_after();
       }
       const float alpha = grow ? ex2(m_ref - mx) : 1.f;
@@ -267,7 +254,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full);
     }
-    if (ok && mbar_wait(&pv_done, (nkv - 1) & 1, abort_v, p.status)) {
+    if (ok && warp_wait(&pv_done, (nkv - 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = qi < p.T;

@@ -1,0 +1,514 @@
+// Weight-absorbed MLA decode on sm_100a (bf16 in, fp32 softmax/accumulation).
+//
+// Megatron-LM MLA guide, 推理优化: each cached token keeps the compressed
+// latent [kv_compressed | k_pos_emb]; decode folds up_k (rows [0, nope) of a
+// head's block of the kv up-projection) into the query and applies up_v
+// (rows [nope, nope+v)) after attention.  Three kernels:
+//
+//   D1 qlat_kernel        q_lat[b,h] = [W_UK[h]^T q_nope[b,h] | q_pe[b,h]]
+//                         (bf16, [B, h, 576]); one block per (head, 256
+//                         latent columns), W read once, fp32 FFMA.
+//   D2 latent_attn_kernel split-KV attention of the 128 heads of a sequence
+//                         over its [ctx, 576] cache, on tcgen05 (below).
+//   D3+D4 combine_vup_kernel  log-sum-exp merge of the splits and
+//                         o[b,h] = W_UV[h] o_lat[b,h]; one block per
+//                         (head, 64 value columns).
+//
+// D2 design.  With 128 heads as the MMA M dimension the latent output
+// O[128, 512] in fp32 fills all 512 TMEM columns, leaving none for the
+// scores.  A cluster of two CTAs therefore shares one (sequence, split):
+// CTA c holds latent columns [256c, 256c+256) of O (256 TMEM columns) and
+// contracts the scores over its share of the 576 cached dims -- CTA 0 over
+// dims [0, 256), CTA 1 over [256, 576) (latent half + the 64 rope dims).
+// Each CTA TMA-loads only its own dims of every 64-token chunk, so every
+// cache byte crosses HBM once; the same shared-memory tile is the K-major B
+// operand of S = Q C^T and the MN-major B operand of O += P C.  The two
+// partial score tiles (fp32, 128 x 64) are exchanged through distributed
+// shared memory; both CTAs add them in the same order and run the identical
+// online softmax, so P, the running max and the row sums agree bit for bit
+// without further exchange.  Warp roles (256 threads per CTA):
+//   warp 0     TMA: Q share once, chunk ring (2 stages), L2 prefetch ahead
+//   warp 1     TMEM allocation, MMA issue (S_j, then O += P_{j-1} C_{j-1})
+//   warps 4-7  score exchange + softmax (thread = head) + epilogue
+// All waits are bounded; a timeout sets the device status word.
+#include <cfloat>
+
+#include "sm100.cuh"
+#include "tc.h"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row width
+constexpr int NT = 64;                           // tokens per chunk
+constexpr int QBOX = 128 * 64 * 2;               // 128 heads x 64 dims bf16
+constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
+constexpr int MAX_ATOMS = 5;
+constexpr int OFF_Q = 0;
+constexpr int OFF_C = OFF_Q + MAX_ATOMS * QBOX;          // 80 KB
+constexpr int STAGE = MAX_ATOMS * CBOX;                  // 40 KB
+constexpr int OFF_X = OFF_C + 2 * STAGE;                 // exchange: 128 x 64 fp32
+constexpr int OFF_P = OFF_X + 128 * NT * 4;              // P: 128 x 64 bf16
+constexpr int SMEM_BYTES = OFF_P + 128 * NT * 2 + 1024;
+constexpr int NTHREADS = 256;
+constexpr int PREFETCH = 4;                              // chunks prefetched to L2
+constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
+constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
+constexpr uint32_t TM_S = 0, TM_O = 256;
+constexpr float kRescaleLog2 = 8.f;
+
+struct DecTcParams {
+  const int32_t* cu_ctx;
+  int B, h, max_ctx;
+  int split_tokens, max_splits;
+  float scale_log2;
+  float* part_o;      // [B, max_splits, h, R]
+  float* part_lse;    // [B, max_splits, h]
+  uint32_t* status;
+};
+
+__device__ __forceinline__ int seq_len(const int32_t* cu, int b, int max_ctx, uint32_t* status,
+                                       int64_t* start) {
+  const int64_t s = cu[b], e = cu[b + 1];
+  int64_t n = e - s;
+  if (n < 1 || n > max_ctx) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusBadCtx);
+    n = n < 1 ? 0 : max_ctx;
+  }
+  *start = s;
+  return (int)n;
+}
+
+// First token (relative to the sequence start) of the 64-row box that chunk j
+// of a split starting at token t0 loads.  A box never reaches past the last
+// token n - 1 of its sequence, so the load stays inside the caller's cache:
+// the last chunk of a sequence is shifted back and its leading tokens, which
+// the previous chunk already covered, are masked.  For n < 64 the box starts
+// before the sequence (rows of earlier sequences, or negative rows that the
+// tensor map fills with zeros); those columns are masked too.
+__device__ __forceinline__ int chunk_base(int n, int t0, int j) {
+  const int lt = t0 + j * NT;
+  return n >= NT ? min(lt, n - NT) : n - NT;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ DecTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full, c_full[2], c_empty[2], s_full[2], s_free[2], p_full,
+      pv_done, x_full, x_empty;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  volatile int* abort_v = &abort_flag;
+
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
+  const int item = blockIdx.x >> 1;
+  const int b = item / p.max_splits, sp = item % p.max_splits;
+  const int h0 = blockIdx.z * 128;
+  int64_t start;
+  const int n = seq_len(p.cu_ctx, b, p.max_ctx, p.status, &start);
+  const int t0 = sp * p.split_tokens;
+  if (t0 >= n) {   // empty split (both CTAs of the pair take this branch)
+    if (rank == 0 && threadIdx.x < 128 && h0 + threadIdx.x < p.h)
+      p.part_lse[((int64_t)b * p.max_splits + sp) * p.h + h0 + threadIdx.x] = -INFINITY;
+    return;
+  }
+  const int tcount = min(p.split_tokens, n - t0);
+  const int nch = (tcount + NT - 1) / NT;
+  const int atoms = rank == 0 ? 4 : 5;
+  const int dim0 = 256 * (int)rank;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&c_full[s], 1);
+      mbar_init(&c_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 4);
+    }
+    mbar_init(&p_full, 4);
+    mbar_init(&pv_done, 1);
+    mbar_init(&x_full, 128);
+    mbar_init(&x_empty, 128);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base, 512);
+    tc_fence_before();
+  }
+  __syncthreads();
+  cluster_sync();          // the peer's barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch(&tmQ);
+      tma_prefetch(&tmC);
+      mbar_arrive_expect_tx(&q_full, atoms * QBOX);
+      for (int a = 0; a < atoms; ++a)
+        tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, dim0 + 64 * a, b * p.h + h0, &q_full);
+      for (int j = 0; j < PREFETCH && j < nch; ++j)
+        for (int a = 0; a < atoms; ++a)
+          tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, (int)start + chunk_base(n, t0, j));
+      for (int j = 0; j < nch; ++j) {
+        const int slot = j & 1;
+        if (j + PREFETCH < nch)
+          for (int a = 0; a < atoms; ++a)
+            tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, (int)start + chunk_base(n, t0, j + PREFETCH));
+        if (!mbar_wait(&c_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
+        uint8_t* sc = smem + OFF_C + slot * STAGE;
+        mbar_arrive_expect_tx(&c_full[slot], atoms * CBOX);
+        const int y = (int)start + chunk_base(n, t0, j);
+        for (int a = 0; a < atoms; ++a)
+          tma_load_2d(sc + a * CBOX, &tmC, dim0 + 64 * a, y, &c_full[slot]);
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      const uint32_t sq = smem_u32(smem + OFF_Q);
+      const uint32_t sp_ = smem_u32(smem + OFF_P);
+      bool ok = mbar_wait(&q_full, 0, abort_v, p.status);
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(&p_full, j & 1, abort_v, p.status)) return false;
+        tc_fence_after();
+        const uint32_t sc = smem_u32(smem + OFF_C + (j & 1) * STAGE);
+#pragma unroll
+        for (int k = 0; k < NT / 16; ++k)
+          mma_bf16(tbase + TM_O, desc_kmajor_sw128(sp_ + k * 32),
+                   desc_mnmajor_sw128(sc + k * 16 * 128, CBOX), IDESC_PV, (j | k) != 0);
+        mma_commit(&c_empty[j & 1]);
+        mma_commit(&pv_done);
+        return true;
+      };
+      for (int j = 0; ok && j < nch; ++j) {
+        const int slot = j & 1;
+        if (!mbar_wait(&c_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
+        if (!mbar_wait(&s_free[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sc = smem_u32(smem + OFF_C + slot * STAGE);
+        for (int a = 0; a < atoms; ++a)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tbase + TM_S + slot * NT, desc_kmajor_sw128(sq + a * QBOX + k * 32),
+                     desc_kmajor_sw128(sc + a * CBOX + k * 32), IDESC_S, (a | k) != 0);
+        mma_commit(&s_full[slot]);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(nch - 1);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;                  // head row within the group
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t sx = smem_u32(smem + OFF_X);
+    const uint32_t sp_ = smem_u32(smem + OFF_P);
+    const uint32_t px = map_peer(sx, peer);
+    const uint32_t px_full = map_peer(smem_u32(&x_full), peer);
+    const uint32_t px_empty = map_peer(smem_u32(&x_empty), peer);
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nch; ++j) {
+      const int slot = j & 1;
+      if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(tbase + lane_off + TM_S + slot * NT, sr[0]);
+      tmem_ld32(tbase + lane_off + TM_S + slot * NT + 32, sr[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[slot]);
+      // exchange the partial scores with the peer CTA (row r, 16 chunks of 4,
+      // chunk position swizzled by the row to spread shared-memory banks)
+      if (!warp_wait_cluster(&x_empty, (j & 1) ^ 1, abort_v, p.status)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int i = c >> 3, e = (c & 7) * 4;
+        st_cluster_v4(px + r * 256 + ((c ^ (r & 15)) << 4), sr[i][e], sr[i][e + 1], sr[i][e + 2],
+                      sr[i][e + 3]);
+      }
+      mbar_arrive_remote(px_full);
+      if (!warp_wait_cluster(&x_full, j & 1, abort_v, p.status)) { ok = false; break; }
+      float s[NT];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        float a0, a1, a2, a3;
+        ld_shared_v4(sx + r * 256 + ((c ^ (r & 15)) << 4), a0, a1, a2, a3);
+        const int i = c >> 3, e = (c & 7) * 4;
+        s[c * 4 + 0] = __uint_as_float(sr[i][e + 0]) + a0;
+        s[c * 4 + 1] = __uint_as_float(sr[i][e + 1]) + a1;
+        s[c * 4 + 2] = __uint_as_float(sr[i][e + 2]) + a2;
+        s[c * 4 + 3] = __uint_as_float(sr[i][e + 3]) + a3;
+      }
+      mbar_arrive_remote(px_empty);
+      // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
+      const int lo = j * NT - (chunk_base(n, t0, j) - t0);
+      const int hi = tcount - (chunk_base(n, t0, j) - t0);
+      float mx = m_ref;
+#pragma unroll
+      for (int i = 0; i < NT; ++i) {
+        s[i] = (i >= lo && i < hi) ? s[i] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+      const bool grow = mx > m_ref + kRescaleLog2;
+      if (j > 0) {
+        if (!warp_wait(&pv_done, (j - 1) & 1, abort_v, p.status)) { ok = false; break; }
+        tc_fence_after();
+      }
+      const float alpha = grow ? ex2(m_ref - mx) : 1.f;
+      if (grow) {
+        l *= alpha;
+        m_ref = mx;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tbase + lane_off + TM_O + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tbase + lane_off + TM_O + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = ex2(s[ch * 8 + 2 * e] - m_ref);
+          const float p1 = ex2(s[ch * 8 + 2 * e + 1] - m_ref);
+          lsum += p0 + p1;
+          w[e] = pack_bf16(p0, p1);
+        }
+        st_shared_v4(sp_ + r * 128 + ((ch ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+      }
+      l += lsum;
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full);
+    }
+    if (ok && warp_wait(&pv_done, (nch - 1) & 1, abort_v, p.status)) {
+      tc_fence_after();
+      const int head = h0 + r;
+      const bool head_ok = head < p.h;
+      const int64_t part = ((int64_t)b * p.max_splits + sp) * p.h + head;
+      const float inv = 1.f / l;
+      float* dst = p.part_o + part * R + dim0;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tbase + lane_off + TM_O + c * 32, o);
+        tmem_wait_ld();
+        if (head_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            st_global_v4(dst + c * 32 + i, __float_as_uint(__uint_as_float(o[i]) * inv),
+                         __float_as_uint(__uint_as_float(o[i + 1]) * inv),
+                         __float_as_uint(__uint_as_float(o[i + 2]) * inv),
+                         __float_as_uint(__uint_as_float(o[i + 3]) * inv));
+        }
+      }
+      if (rank == 0 && head_ok) p.part_lse[part] = (m_ref + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();          // the peer no longer touches this CTA's shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// D1: q_lat = [W_UK^T q_nope | q_pe] for up to 64 sequences per pass.
+__global__ void __launch_bounds__(256)
+    qlat_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* __restrict__ q_pe,
+                const __nv_bfloat16* __restrict__ w_kv_b, __nv_bfloat16* __restrict__ q_lat,
+                int B, int h, int dn, int dv) {
+  extern __shared__ float qn[];                      // [64][dn]
+  const int hh = blockIdx.x;
+  const int c = blockIdx.y * 256 + threadIdx.x;      // latent column
+  const __nv_bfloat16* wk = w_kv_b + (int64_t)hh * (dn + dv) * R;
+  for (int b0 = 0; b0 < B; b0 += 64) {
+    const int nb = min(64, B - b0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb * dn; i += blockDim.x) {
+      const int bb = i / dn, d = i % dn;
+      qn[bb * dn + d] = __bfloat162float(q_nope[((int64_t)(b0 + bb) * h + hh) * dn + d]);
+    }
+    __syncthreads();
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    for (int d = 0; d < dn; ++d) {
+      const float w = __bfloat162float(wk[(int64_t)d * R + c]);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = fmaf(qn[i * dn + d], w, acc[i]);
+    }
+    for (int i = 0; i < nb; ++i)
+      q_lat[((int64_t)(b0 + i) * h + hh) * W + c] = __float2bfloat16_rn(acc[i]);
+    if (blockIdx.y == 0 && threadIdx.x < DR)
+      for (int i = 0; i < nb; ++i)
+        q_lat[((int64_t)(b0 + i) * h + hh) * W + R + threadIdx.x] =
+            q_pe[((int64_t)(b0 + i) * h + hh) * DR + threadIdx.x];
+  }
+}
+
+// D3 + D4: o[b,h,v] = W_UV[h][v] . sum_s w_s part_o[b,s,h], w_s = exp(lse_s - lse) .
+// One block per (head, 64 value columns); W_UV slice staged transposed.
+__global__ void __launch_bounds__(256)
+    combine_vup_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                       const __nv_bfloat16* __restrict__ w_kv_b, __nv_bfloat16* __restrict__ o,
+                       int B, int h, int dn, int dv, int max_splits) {
+  extern __shared__ float sm[];
+  float* wt = sm;                    // [R][64]  W_UV[h][v0 + v][r] transposed
+  float* ol = wt + R * 64;           // [16][R]  merged latent outputs of 16 sequences
+  __shared__ float wgt[16][64];      // split weights
+  const int hh = blockIdx.x, v0 = blockIdx.y * 64;
+  const __nv_bfloat16* wv = w_kv_b + ((int64_t)hh * (dn + dv) + dn + v0) * R;
+  for (int i = threadIdx.x; i < 64 * R; i += blockDim.x) {
+    const int v = i / R, c = i % R;
+    wt[c * 64 + v] = v0 + v < dv ? __bfloat162float(wv[(int64_t)v * R + c]) : 0.f;
+  }
+  const int v = threadIdx.x % 64, g = threadIdx.x / 64;    // 4 groups x 4 sequences
+  for (int b0 = 0; b0 < B; b0 += 16) {
+    const int nb = min(16, B - b0);
+    __syncthreads();
+    if (threadIdx.x < 16) {
+      const int bb = threadIdx.x;
+      if (bb < nb) {
+        const float* lse = part_lse + (int64_t)(b0 + bb) * max_splits * h + hh;
+        float mx = -INFINITY;
+        for (int s = 0; s < max_splits; ++s) mx = fmaxf(mx, lse[(int64_t)s * h]);
+        float den = 0.f;
+        for (int s = 0; s < max_splits; ++s) {
+          const float x = lse[(int64_t)s * h];
+          const float e = x == -INFINITY ? 0.f : __expf(x - mx);
+          wgt[bb][s < 64 ? s : 63] = e;
+          den += e;
+        }
+        for (int s = 0; s < max_splits && s < 64; ++s) wgt[bb][s] = den > 0.f ? wgt[bb][s] / den : 0.f;
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb * R; i += blockDim.x) {
+      const int bb = i / R, c = i % R;
+      float acc = 0.f;
+      for (int s = 0; s < max_splits; ++s) {
+        const float w = wgt[bb][s];
+        if (w != 0.f) acc = fmaf(w, part_o[(((int64_t)(b0 + bb) * max_splits + s) * h + hh) * R + c], acc);
+      }
+      ol[bb * R + c] = acc;
+    }
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < R; ++c) {
+      const float w = wt[c * 64 + v];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = fmaf(w, ol[(g * 4 + k) * R + c], acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int bb = g * 4 + k;
+      if (bb < nb && v0 + v < dv)
+        o[((int64_t)(b0 + bb) * h + hh) * dv + v0 + v] = __float2bfloat16_rn(acc[k]);
+    }
+  }
+}
+
+}  // namespace
+
+bool tc_decode_supported(const mla_config& c) {
+  return c.dtype == MLA_BF16 && c.kv_lora_rank == R && c.qk_rope_head_dim == DR &&
+         c.qk_nope_head_dim <= 256 && c.v_head_dim % 64 == 0;
+}
+
+int tc_decode_split_tokens() { return 4096; }
+
+cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
+  // D1
+  {
+    const size_t smem = 64 * a.dn * sizeof(float);
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(qlat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    qlat_kernel<<<dim3(a.h, R / 256), 256, smem, st>>>(
+        (const __nv_bfloat16*)a.q_nope, (const __nv_bfloat16*)a.q_pe,
+        (const __nv_bfloat16*)a.w_kv_b, (__nv_bfloat16*)a.q_lat, a.B, a.h, a.dn, a.dv);
+    count_launches();
+  }
+  stage_event(1, st);
+  // D2
+  {
+    CUtensorMap tmQ, tmC;
+    const uint32_t qbox[2] = {64, 128}, cbox[2] = {64, NT};
+    const uint64_t qdims[2] = {(uint64_t)W, (uint64_t)a.B * a.h};
+    const uint64_t qstr[1] = {(uint64_t)W * 2};
+    if (!encode_tmap(&tmQ, a.q_lat, 2, qdims, qstr, qbox)) return cudaErrorInvalidValue;
+    // The cache holds sum(ctx) <= B * max_ctx rows; cu_ctx lives on the
+    // device, so the map is declared with the bound and every box is clamped
+    // inside its own sequence (chunk_base).
+    const uint64_t cdims[2] = {(uint64_t)W, (uint64_t)a.B * (uint64_t)a.max_ctx};
+    const uint64_t cstr[1] = {(uint64_t)W * 2};
+    if (!encode_tmap(&tmC, a.cache, 2, cdims, cstr, cbox)) return cudaErrorInvalidValue;
+    DecTcParams p{};
+    p.cu_ctx = a.cu_ctx;
+    p.B = a.B;
+    p.h = a.h;
+    p.max_ctx = a.max_ctx;
+    p.split_tokens = a.split_tokens;
+    p.max_splits = a.max_splits;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.part_o = a.part_o;
+    p.part_lse = a.part_lse;
+    p.status = a.status;
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    dim3 grid(2 * a.B * a.max_splits, 1, (a.h + 127) / 128);
+    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmC, p);
+    count_launches();
+  }
+  stage_event(2, st);
+  stage_event(3, st);
+  // D3 + D4
+  {
+    const size_t smem = (size_t)(R * 64 + 16 * R) * sizeof(float);
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(combine_vup_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    combine_vup_kernel<<<dim3(a.h, (a.dv + 63) / 64), 256, smem, st>>>(
+        a.part_o, a.part_lse, (const __nv_bfloat16*)a.w_kv_b, (__nv_bfloat16*)a.o, a.B, a.h,
+        a.dn, a.dv, a.max_splits);
+    count_launches();
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
       const uint32_t tph = (local >> 1) & 1;
-      if (!mbar_wait(&tfull[buf], tph, abort_v, p.status)) break;
+      if (!warp_wait(&tfull[buf], tph, abort_v, p.status)) break;
       tc_fence_after();
       int s, m0, n0;
       tile_coords(p, t, s, m0, n0);
