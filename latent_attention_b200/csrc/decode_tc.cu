@@ -5,14 +5,13 @@
 // head's block of the kv up-projection) into the query and applies up_v
 // (rows [nope, nope+v)) after attention.  Three kernels:
 //
-//   D1 qlat_kernel        q_lat[b,h] = [W_UK[h]^T q_nope[b,h] | q_pe[b,h]]
-//                         (bf16, [B, h, 576]); one block per (head, 256
-//                         latent columns), W read once, fp32 FFMA.
-//   D2 latent_attn_kernel split-KV attention of the 128 heads of a sequence
-//                         over its [ctx, 576] cache, on tcgen05 (below).
-//   D3+D4 combine_vup_kernel  log-sum-exp merge of the splits and
-//                         o[b,h] = W_UV[h] o_lat[b,h]; one block per
-//                         (head, 64 value columns).
+//   D1 q_lat[b,h] = W_UK[h]^T q_nope[b,h]          batched tcgen05 GEMM (one
+//                                                   product per head, W_UK read
+//                                                   as an MN-major operand)
+//   D2 latent_attn_kernel  split-KV attention of the 128 heads of a sequence
+//                          over its [ctx, 576] cache, on tcgen05 (below)
+//   D3 combine_kernel      log-sum-exp merge of the splits -> o_lat (bf16)
+//   D4 o[b,h] = W_UV[h] o_lat[b,h]                  batched tcgen05 GEMM
 //
 // D2 design.  With 128 heads as the MMA M dimension the latent output
 // O[128, 512] in fp32 fills all 512 TMEM columns, leaving none for the
@@ -95,6 +94,7 @@ __device__ __forceinline__ int chunk_base(int n, int t0, int j) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmQpe,
                        const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -135,7 +135,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(&p_full, 4);
     mbar_init(&pv_done, 1);
-    mbar_init(&x_full, 128);
+    mbar_init(&x_full, 1);     // one local arrive.expect_tx + the peer's st.async bytes
     mbar_init(&x_empty, 128);
     abort_flag = 0;
     fence_barrier_init();
@@ -152,10 +152,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     if (elect_one()) {
       tma_prefetch(&tmQ);
+      tma_prefetch(&tmQpe);
       tma_prefetch(&tmC);
       mbar_arrive_expect_tx(&q_full, atoms * QBOX);
-      for (int a = 0; a < atoms; ++a)
+      for (int a = 0; a < 4; ++a)
         tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, dim0 + 64 * a, b * p.h + h0, &q_full);
+      if (atoms == 5)
+        tma_load_2d(smem + OFF_Q + 4 * QBOX, &tmQpe, 0, b * p.h + h0, &q_full);
       for (int j = 0; j < PREFETCH && j < nch; ++j)
         for (int a = 0; a < atoms; ++a)
           tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, (int)start + chunk_base(n, t0, j));
@@ -233,10 +236,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const int i = c >> 3, e = (c & 7) * 4;
-        st_cluster_v4(px + r * 256 + ((c ^ (r & 15)) << 4), sr[i][e], sr[i][e + 1], sr[i][e + 2],
-                      sr[i][e + 3]);
+        st_async_v4(px + r * 256 + ((c ^ (r & 15)) << 4), sr[i][e], sr[i][e + 1], sr[i][e + 2],
+                    sr[i][e + 3], px_full);
       }
-      mbar_arrive_remote(px_full);
+      if (r == 0) mbar_arrive_expect_tx(&x_full, 128 * NT * 4);
       if (!warp_wait_cluster(&x_full, j & 1, abort_v, p.status)) { ok = false; break; }
       float s[NT];
 #pragma unroll
@@ -334,135 +337,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// D1: q_lat = [W_UK^T q_nope | q_pe] for up to 64 sequences per pass.
-__global__ void __launch_bounds__(256)
-    qlat_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* __restrict__ q_pe,
-                const __nv_bfloat16* __restrict__ w_kv_b, __nv_bfloat16* __restrict__ q_lat,
-                int B, int h, int dn, int dv) {
-  extern __shared__ float qn[];                      // [64][dn]
-  const int hh = blockIdx.x;
-  const int c = blockIdx.y * 256 + threadIdx.x;      // latent column
-  const __nv_bfloat16* wk = w_kv_b + (int64_t)hh * (dn + dv) * R;
-  for (int b0 = 0; b0 < B; b0 += 64) {
-    const int nb = min(64, B - b0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < nb * dn; i += blockDim.x) {
-      const int bb = i / dn, d = i % dn;
-      qn[bb * dn + d] = __bfloat162float(q_nope[((int64_t)(b0 + bb) * h + hh) * dn + d]);
-    }
-    __syncthreads();
-    float acc[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-    for (int d = 0; d < dn; ++d) {
-      const float w = __bfloat162float(wk[(int64_t)d * R + c]);
-#pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = fmaf(qn[i * dn + d], w, acc[i]);
-    }
-    for (int i = 0; i < nb; ++i)
-      q_lat[((int64_t)(b0 + i) * h + hh) * W + c] = __float2bfloat16_rn(acc[i]);
-    if (blockIdx.y == 0 && threadIdx.x < DR)
-      for (int i = 0; i < nb; ++i)
-        q_lat[((int64_t)(b0 + i) * h + hh) * W + R + threadIdx.x] =
-            q_pe[((int64_t)(b0 + i) * h + hh) * DR + threadIdx.x];
+// D3: o_lat[b,h] = sum_s w_s part_o[b,s,h] with w_s = exp(lse_s - max) / sum,
+// one block per (sequence, head), 4 latent columns per thread.
+__global__ void __launch_bounds__(128)
+    combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                   __nv_bfloat16* __restrict__ o_lat, int h, int max_splits) {
+  const int b = blockIdx.x / h, hh = blockIdx.x % h;
+  const int c = threadIdx.x * 4;
+  const float* lse = part_lse + (int64_t)b * max_splits * h + hh;
+  float mx = -INFINITY;
+  for (int s = 0; s < max_splits; ++s) mx = fmaxf(mx, lse[(int64_t)s * h]);
+  float den = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < max_splits; ++s) {
+    const float l = lse[(int64_t)s * h];
+    if (l == -INFINITY) continue;
+    const float w = __expf(l - mx);
+    const float4 v = *reinterpret_cast<const float4*>(
+        part_o + (((int64_t)b * max_splits + s) * h + hh) * R + c);
+    den += w;
+    a0 = fmaf(w, v.x, a0);
+    a1 = fmaf(w, v.y, a1);
+    a2 = fmaf(w, v.z, a2);
+    a3 = fmaf(w, v.w, a3);
   }
-}
-
-// D3 + D4: o[b,h,v] = W_UV[h][v] . sum_s w_s part_o[b,s,h], w_s = exp(lse_s - lse) .
-// One block per (head, 64 value columns); W_UV slice staged transposed.
-__global__ void __launch_bounds__(256)
-    combine_vup_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                       const __nv_bfloat16* __restrict__ w_kv_b, __nv_bfloat16* __restrict__ o,
-                       int B, int h, int dn, int dv, int max_splits) {
-  extern __shared__ float sm[];
-  float* wt = sm;                    // [R][64]  W_UV[h][v0 + v][r] transposed
-  float* ol = wt + R * 64;           // [16][R]  merged latent outputs of 16 sequences
-  __shared__ float wgt[16][64];      // split weights
-  const int hh = blockIdx.x, v0 = blockIdx.y * 64;
-  const __nv_bfloat16* wv = w_kv_b + ((int64_t)hh * (dn + dv) + dn + v0) * R;
-  for (int i = threadIdx.x; i < 64 * R; i += blockDim.x) {
-    const int v = i / R, c = i % R;
-    wt[c * 64 + v] = v0 + v < dv ? __bfloat162float(wv[(int64_t)v * R + c]) : 0.f;
-  }
-  const int v = threadIdx.x % 64, g = threadIdx.x / 64;    // 4 groups x 4 sequences
-  for (int b0 = 0; b0 < B; b0 += 16) {
-    const int nb = min(16, B - b0);
-    __syncthreads();
-    if (threadIdx.x < 16) {
-      const int bb = threadIdx.x;
-      if (bb < nb) {
-        const float* lse = part_lse + (int64_t)(b0 + bb) * max_splits * h + hh;
-        float mx = -INFINITY;
-        for (int s = 0; s < max_splits; ++s) mx = fmaxf(mx, lse[(int64_t)s * h]);
-        float den = 0.f;
-        for (int s = 0; s < max_splits; ++s) {
-          const float x = lse[(int64_t)s * h];
-          const float e = x == -INFINITY ? 0.f : __expf(x - mx);
-          wgt[bb][s < 64 ? s : 63] = e;
-          den += e;
-        }
-        for (int s = 0; s < max_splits && s < 64; ++s) wgt[bb][s] = den > 0.f ? wgt[bb][s] / den : 0.f;
-      }
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < nb * R; i += blockDim.x) {
-      const int bb = i / R, c = i % R;
-      float acc = 0.f;
-      for (int s = 0; s < max_splits; ++s) {
-        const float w = wgt[bb][s];
-        if (w != 0.f) acc = fmaf(w, part_o[(((int64_t)(b0 + bb) * max_splits + s) * h + hh) * R + c], acc);
-      }
-      ol[bb * R + c] = acc;
-    }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < R; ++c) {
-      const float w = wt[c * 64 + v];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = fmaf(w, ol[(g * 4 + k) * R + c], acc[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int bb = g * 4 + k;
-      if (bb < nb && v0 + v < dv)
-        o[((int64_t)(b0 + bb) * h + hh) * dv + v0 + v] = __float2bfloat16_rn(acc[k]);
-    }
-  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  __nv_bfloat16* dst = o_lat + ((int64_t)b * h + hh) * R + c;
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(a0 * inv, a1 * inv),
+                                              pack_bf16(a2 * inv, a3 * inv));
 }
 
 }  // namespace
 
 bool tc_decode_supported(const mla_config& c) {
   return c.dtype == MLA_BF16 && c.kv_lora_rank == R && c.qk_rope_head_dim == DR &&
-         c.qk_nope_head_dim <= 256 && c.v_head_dim % 64 == 0;
+         c.qk_nope_head_dim % 8 == 0 && c.v_head_dim % 8 == 0;
 }
 
 int tc_decode_split_tokens() { return 4096; }
 
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
-  // D1
+  cudaError_t e;
+  // D1: q_lat[b, h, :] = q_nope[b, h, :] W_UK[h]  (per head: [B, dn] x [dn, R])
   {
-    const size_t smem = 64 * a.dn * sizeof(float);
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(qlat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    qlat_kernel<<<dim3(a.h, R / 256), 256, smem, st>>>(
-        (const __nv_bfloat16*)a.q_nope, (const __nv_bfloat16*)a.q_pe,
-        (const __nv_bfloat16*)a.w_kv_b, (__nv_bfloat16*)a.q_lat, a.B, a.h, a.dn, a.dv);
-    count_launches();
+    GemmArgs g;
+    g.A = a.q_nope; g.lda = (int64_t)a.h * a.dn; g.sA = a.dn; g.a_batch_inner = true;
+    g.Bm[0] = a.w_kv_b; g.ldb[0] = R; g.sB = (int64_t)(a.dn + a.dv) * R; g.b_mn = true;
+    g.M = a.B; g.K = a.dn; g.batch = a.h; g.nseg = 1;
+    g.seg[0].out = a.q_lat; g.seg[0].ldo = (int64_t)a.h * R; g.seg[0].ncols = R;
+    g.sOut = R;
+    if (!tc_gemm_supported(g, MLA_BF16)) return cudaErrorNotSupported;
+    e = tc_gemm(g, st, a.status);
+    if (e != cudaSuccess) return e;
   }
   stage_event(1, st);
   // D2
   {
-    CUtensorMap tmQ, tmC;
+    CUtensorMap tmQ, tmQpe, tmC;
     const uint32_t qbox[2] = {64, 128}, cbox[2] = {64, NT};
-    const uint64_t qdims[2] = {(uint64_t)W, (uint64_t)a.B * a.h};
-    const uint64_t qstr[1] = {(uint64_t)W * 2};
+    const uint64_t qdims[2] = {(uint64_t)R, (uint64_t)a.B * a.h};
+    const uint64_t qstr[1] = {(uint64_t)R * 2};
     if (!encode_tmap(&tmQ, a.q_lat, 2, qdims, qstr, qbox)) return cudaErrorInvalidValue;
+    const uint64_t pdims[2] = {(uint64_t)DR, (uint64_t)a.B * a.h};
+    const uint64_t pstr[1] = {(uint64_t)DR * 2};
+    if (!encode_tmap(&tmQpe, a.q_pe, 2, pdims, pstr, qbox)) return cudaErrorInvalidValue;
     // The cache holds sum(ctx) <= B * max_ctx rows; cu_ctx lives on the
     // device, so the map is declared with the bound and every box is clamped
     // inside its own sequence (chunk_base).
@@ -482,31 +420,35 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
     p.status = a.status;
     static bool attr = false;
     if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      e = cudaFuncSetAttribute(latent_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMEM_BYTES);
       if (e != cudaSuccess) return e;
       attr = true;
     }
     dim3 grid(2 * a.B * a.max_splits, 1, (a.h + 127) / 128);
-    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmC, p);
+    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, p);
     count_launches();
   }
   stage_event(2, st);
+  // D3
+  combine_kernel<<<a.B * a.h, R / 4, 0, st>>>(a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat,
+                                              a.h, a.max_splits);
+  count_launches();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   stage_event(3, st);
-  // D3 + D4
+  // D4: o[b, h, :] = o_lat[b, h, :] W_UV[h]^T  (per head: [B, R] x [R, dv])
   {
-    const size_t smem = (size_t)(R * 64 + 16 * R) * sizeof(float);
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(combine_vup_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    combine_vup_kernel<<<dim3(a.h, (a.dv + 63) / 64), 256, smem, st>>>(
-        a.part_o, a.part_lse, (const __nv_bfloat16*)a.w_kv_b, (__nv_bfloat16*)a.o, a.B, a.h,
-        a.dn, a.dv, a.max_splits);
-    count_launches();
+    GemmArgs g;
+    g.A = a.o_lat; g.lda = (int64_t)a.h * R; g.sA = R; g.a_batch_inner = true;
+    g.Bm[0] = reinterpret_cast<const __nv_bfloat16*>(a.w_kv_b) + (int64_t)a.dn * R;
+    g.ldb[0] = R; g.sB = (int64_t)(a.dn + a.dv) * R;
+    g.M = a.B; g.K = R; g.batch = a.h; g.nseg = 1;
+    g.seg[0].out = a.o; g.seg[0].ldo = (int64_t)a.h * a.dv; g.seg[0].ncols = a.dv;
+    g.sOut = a.dv;
+    if (!tc_gemm_supported(g, MLA_BF16)) return cudaErrorNotSupported;
+    e = tc_gemm(g, st, a.status);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -5,6 +5,10 @@
 // segments with their own B matrix (the fused q_a | kv_a down-projection of
 // the CSDN DeepseekV3Attention forward shares the input x).
 //
+// Batched products (one per head, for the absorbed decode) index a third
+// tensor-map dimension; a B stored [K, N] (the up_k slice of the kv
+// up-projection) is loaded as four 64-column MN-major boxes per stage.
+//
 // Persistent, warp-specialised kernel, one CTA per SM:
 //   warp 0      TMA producer: 128x64 A box + 256x64 B box per stage,
 //               128-byte swizzle, 4-stage ring of mbarriers
@@ -30,6 +34,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
 constexpr int NTHREADS = 192;
 constexpr uint32_t IDESC = idesc_bf16(BM, BN);
+constexpr uint32_t IDESC_BMN = idesc_bf16(BM, BN, 0, 1);
+constexpr int BMN_BOX = 64 * BK * 2;       // one 64-column MN-major box of B
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
 struct TcGemmParams {
@@ -37,13 +43,18 @@ struct TcGemmParams {
   int nseg;
   int tiles_m;
   int tiles_n[2];
+  int per_batch;          // tiles of one batch entry
   int total_tiles;
+  int a_batch_inner, b_mn;
+  int64_t sOut;
   EpiSeg seg[2];
   uint32_t* status;
 };
 
-__device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& s, int& m0,
-                                            int& n0) {
+__device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& bi, int& s,
+                                            int& m0, int& n0) {
+  bi = t / p.per_batch;
+  t -= bi * p.per_batch;
   const int first = p.tiles_m * p.tiles_n[0];
   s = (t >= first) ? 1 : 0;
   const int local = s ? t - first : t;
@@ -52,8 +63,8 @@ __device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& s
 }
 
 // Epilogue of one 128 x BN tile; this thread owns output row m0 + row.
-__device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSeg& e, int m0,
-                                              int n0, int row, uint32_t taddr) {
+__device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSeg& e, int bi,
+                                              int m0, int n0, int row, uint32_t taddr) {
   const int m = m0 + row;
   const bool row_ok = m < p.M;
   float rs = 1.f;
@@ -64,7 +75,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
   }
   const int pos = row_ok ? m % e.T : 0;
   float ssq = 0.f;
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out);
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out) + (int64_t)bi * p.sOut;
   const __nv_bfloat16* gamma = reinterpret_cast<const __nv_bfloat16*>(e.gamma);
 #pragma unroll 1
   for (int g = 0; g < BN / 64; ++g) {
@@ -172,15 +183,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-        int s, m0, n0;
-        tile_coords(p, t, s, m0, n0);
+        int bi, s, m0, n0;
+        tile_coords(p, t, bi, s, m0, n0);
         const CUtensorMap* tmB = s ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_v, p.status)) goto done;
           uint8_t* sa = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, kb * BK, m0, &full[stage]);
-          tma_load_2d(sa + A_BYTES, tmB, kb * BK, n0, &full[stage]);
+          if (p.a_batch_inner)
+            tma_load_3d(sa, &tmA, kb * BK, bi, m0, &full[stage]);
+          else
+            tma_load_3d(sa, &tmA, kb * BK, m0, bi, &full[stage]);
+          if (p.b_mn) {
+            for (int q = 0; q < BN / 64; ++q)
+              tma_load_3d(sa + A_BYTES + q * BMN_BOX, tmB, n0 + 64 * q, kb * BK, bi, &full[stage]);
+          } else {
+            tma_load_3d(sa + A_BYTES, tmB, kb * BK, n0, bi, &full[stage]);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -204,10 +223,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
+          if (p.b_mn) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_bf16(d, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), IDESC,
-                     (kb | k) != 0);
+            for (int k = 0; k < BK / 16; ++k)
+              mma_bf16(d, desc_kmajor_sw128(sa + k * 32),
+                       desc_mnmajor_sw128(sb + k * 16 * 128, BMN_BOX), IDESC_BMN, (kb | k) != 0);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              mma_bf16(d, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), IDESC,
+                       (kb | k) != 0);
+          }
           mma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -226,9 +252,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t tph = (local >> 1) & 1;
       if (!warp_wait(&tfull[buf], tph, abort_v, p.status)) break;
       tc_fence_after();
-      int s, m0, n0;
-      tile_coords(p, t, s, m0, n0);
-      epilogue_tile(p, p.seg[s], m0, n0, row, tbase + ((uint32_t)(quad * 32) << 16) + buf * BN);
+      int bi, s, m0, n0;
+      tile_coords(p, t, bi, s, m0, n0);
+      epilogue_tile(p, p.seg[s], bi, m0, n0, row,
+                    tbase + ((uint32_t)(quad * 32) << 16) + buf * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -259,12 +286,15 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 bool tc_gemm_supported(const GemmArgs& a, int dtype) {
-  if (dtype != MLA_BF16 || a.M < 1 || a.K < 1) return false;
-  if (a.K % 8 || a.lda % 8 || !aligned16(a.A)) return false;
+  if (dtype != MLA_BF16 || a.M < 1 || a.K < 1 || a.batch < 1) return false;
+  if (a.K % 8 || a.lda % 8 || a.sA % 8 || a.sB % 8 || !aligned16(a.A)) return false;
+  if (a.batch > 1 && (a.nseg != 1 || a.seg[0].ssq_out || a.seg[0].ssq_in || a.seg[0].cos))
+    return false;
   for (int s = 0; s < a.nseg; ++s) {
     const EpiSeg& e = a.seg[s];
     if (a.ldb[s] % 8 || !aligned16(a.Bm[s]) || !aligned16(e.out)) return false;
     if (e.ncols < 1 || e.ncols % 8 || e.ldo % 8) return false;
+    if (a.b_mn && e.ncols % 64) return false;
     if (e.cos && (e.rope_dim != 64 || e.rope_start % 64 || e.rope_period % 64)) return false;
     if (e.ssq_in && e.ssq_parts < 1) return false;
   }
@@ -273,31 +303,57 @@ bool tc_gemm_supported(const GemmArgs& a, int dtype) {
 
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   CUtensorMap tmA, tmB[2];
+  const uint64_t nb = (uint64_t)a.batch;
   {
-    const uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
-    const uint64_t strides[1] = {(uint64_t)a.lda * 2};
-    const uint32_t box[2] = {BK, BM};
-    if (!encode_tmap(&tmA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    // 3D map ordered so that strides grow: {K, rows, batch} or {K, batch, rows}
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    if (a.a_batch_inner) {
+      dims[0] = a.K; dims[1] = nb; dims[2] = a.M;
+      strides[0] = (uint64_t)a.sA * 2; strides[1] = (uint64_t)a.lda * 2;
+      box[0] = BK; box[1] = 1; box[2] = BM;
+    } else {
+      dims[0] = a.K; dims[1] = a.M; dims[2] = nb;
+      strides[0] = (uint64_t)a.lda * 2;
+      strides[1] = a.batch > 1 ? (uint64_t)a.sA * 2 : (uint64_t)a.lda * 2 * a.M;
+      box[0] = BK; box[1] = BM; box[2] = 1;
+    }
+    if (!encode_tmap(&tmA, a.A, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   TcGemmParams p{};
   p.M = a.M;
   p.K = a.K;
   p.nseg = a.nseg;
   p.tiles_m = (a.M + BM - 1) / BM;
-  p.total_tiles = 0;
+  p.per_batch = 0;
   for (int s = 0; s < a.nseg; ++s) {
-    const uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.seg[s].ncols};
-    const uint64_t strides[1] = {(uint64_t)a.ldb[s] * 2};
-    const uint32_t box[2] = {BK, BN};
-    if (!encode_tmap(&tmB[s], a.Bm[s], 2, dims, strides, box)) return cudaErrorInvalidValue;
+    const int64_t n = a.seg[s].ncols;
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    if (a.b_mn) {   // B stored [K, N]
+      dims[0] = n; dims[1] = a.K; dims[2] = nb;
+      strides[0] = (uint64_t)a.ldb[s] * 2;
+      strides[1] = a.batch > 1 ? (uint64_t)a.sB * 2 : (uint64_t)a.ldb[s] * 2 * a.K;
+      box[0] = 64; box[1] = BK; box[2] = 1;
+    } else {        // B stored [N, K]
+      dims[0] = a.K; dims[1] = n; dims[2] = nb;
+      strides[0] = (uint64_t)a.ldb[s] * 2;
+      strides[1] = a.batch > 1 ? (uint64_t)a.sB * 2 : (uint64_t)a.ldb[s] * 2 * n;
+      box[0] = BK; box[1] = BN; box[2] = 1;
+    }
+    if (!encode_tmap(&tmB[s], a.Bm[s], 3, dims, strides, box)) return cudaErrorInvalidValue;
     p.seg[s] = a.seg[s];
-    p.tiles_n[s] = (a.seg[s].ncols + BN - 1) / BN;
-    p.total_tiles += p.tiles_m * p.tiles_n[s];
+    p.tiles_n[s] = (int)((n + BN - 1) / BN);
+    p.per_batch += p.tiles_m * p.tiles_n[s];
   }
   if (a.nseg == 1) {
     tmB[1] = tmB[0];
     p.tiles_n[1] = 0;
   }
+  p.total_tiles = p.per_batch * a.batch;
+  p.a_batch_inner = a.a_batch_inner;
+  p.b_mn = a.b_mn;
+  p.sOut = a.sOut;
   p.status = status;
   static bool attr = false;
   if (!attr) {

@@ -58,6 +58,12 @@ struct EpiSeg {
 
 // C = A B^T with A [M, K] (row stride lda) and the output columns split in up
 // to two segments: columns of segment s come from rows of Bs [ncols_s, K].
+//
+// Batched products (one per attention head in decode): batch i reads
+// A + i*sA, B + i*sB and writes out + i*sOut (elements).  a_batch_inner marks
+// an A whose batch stride is smaller than its row stride ([rows, batch, K]
+// storage).  b_mn marks a B stored [K, N] (N contiguous, row stride ldb)
+// instead of nn.Linear's [N, K].
 struct GemmArgs {
   const void* A = nullptr;
   int64_t lda = 0;
@@ -66,6 +72,10 @@ struct GemmArgs {
   int M = 0, K = 0;
   int nseg = 1;
   EpiSeg seg[2];
+  int batch = 1;
+  int64_t sA = 0, sB = 0, sOut = 0;
+  bool a_batch_inner = false;
+  bool b_mn = false;
 };
 
 struct AttnArgs {
