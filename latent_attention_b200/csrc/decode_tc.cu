@@ -31,6 +31,7 @@
 //   warps 4-7  score exchange + softmax (thread = head) + epilogue
 // All waits are bounded; a timeout sets the device status word.
 #include <cfloat>
+#include <cuda_fp16.h>
 
 #include "sm100.cuh"
 #include "tc.h"
@@ -48,10 +49,10 @@ constexpr int MAX_ATOMS = 5;
 constexpr int OFF_Q = 0;
 constexpr int OFF_C = OFF_Q + MAX_ATOMS * QBOX;          // 80 KB
 constexpr int STAGE = MAX_ATOMS * CBOX;                  // 40 KB
-constexpr int OFF_X = OFF_C + 2 * STAGE;                 // exchange: 128 x 64 fp32
-constexpr int OFF_P = OFF_X + 128 * NT * 4;              // P: 128 x 64 bf16
+constexpr int OFF_X = OFF_C + 2 * STAGE;                 // exchange: 128 x 64 fp16
+constexpr int OFF_P = OFF_X + 128 * NT * 2;              // P: 128 x 64 bf16
 constexpr int SMEM_BYTES = OFF_P + 128 * NT * 2 + 1024;
-constexpr int NTHREADS = 256;
+constexpr int NTHREADS = 320;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
@@ -92,14 +93,23 @@ __device__ __forceinline__ int chunk_base(int n, int t0, int j) {
   return n >= NT ? min(lt, n - NT) : n - NT;
 }
 
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_half2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2*>(&v));
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmQpe,
                        const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, c_full[2], c_empty[2], s_full[2], s_free[2], p_full,
-      pv_done, x_full, x_empty;
+  __shared__ __align__(8) uint64_t q_full, c_full[2], c_empty[2], s_full[2], s_comb[2],
+      s_free[2], p_full, pv_done, x_full, x_empty;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -131,12 +141,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&c_full[s], 1);
       mbar_init(&c_empty[s], 1);
       mbar_init(&s_full[s], 1);
+      mbar_init(&s_comb[s], 4);
       mbar_init(&s_free[s], 4);
     }
     mbar_init(&p_full, 4);
     mbar_init(&pv_done, 1);
     mbar_init(&x_full, 1);     // one local arrive.expect_tx + the peer's st.async bytes
-    mbar_init(&x_empty, 128);
+    mbar_init(&x_empty, 4);    // one arrive per exchange warp of the peer
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -148,6 +159,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   cluster_sync();          // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tbase = tmem_base;
+  // exchange warps 2, 3, 8, 9 and softmax warps 4..7 each cover TMEM lane
+  // quarter (warp & 3), i.e. heads 32 * (warp & 3) .. + 31.
+  const bool xwg = warp == 2 || warp == 3 || warp == 8 || warp == 9;
 
   if (warp == 0) {
     if (elect_one()) {
@@ -208,20 +222,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       if (ok) issue_pv(nch - 1);
     }
-  } else if (warp >= 4) {
+  } else if (xwg) {
+    // ---------------- score exchange: own partial (fp16) to the peer, peer's
+    // partial back, merged scores (fp32) written over the TMEM slot.
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;                  // head row within the group
+    const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t sx = smem_u32(smem + OFF_X);
-    const uint32_t sp_ = smem_u32(smem + OFF_P);
     const uint32_t px = map_peer(sx, peer);
     const uint32_t px_full = map_peer(smem_u32(&x_full), peer);
     const uint32_t px_empty = map_peer(smem_u32(&x_empty), peer);
+    for (int j = 0; j < nch; ++j) {
+      const int slot = j & 1;
+      if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) break;
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(tbase + lane_off + TM_S + slot * NT, sr[0]);
+      tmem_ld32(tbase + lane_off + TM_S + slot * NT + 32, sr[1]);
+      tmem_wait_ld();
+      uint32_t h[32];                                 // own partial as fp16 pairs
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        h[i] = pack_half2(__uint_as_float(sr[i >> 4][(2 * i) & 31]),
+                          __uint_as_float(sr[i >> 4][(2 * i + 1) & 31]));
+      if (!warp_wait_cluster(&x_empty, (j & 1) ^ 1, abort_v, p.status)) break;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_async_v4(px + r * 128 + ((c ^ (r & 7)) << 4), h[4 * c], h[4 * c + 1], h[4 * c + 2],
+                    h[4 * c + 3], px_full);
+      if (r == 0) mbar_arrive_expect_tx(&x_full, 128 * NT * 2);
+      if (!warp_wait_cluster(&x_full, j & 1, abort_v, p.status)) break;
+      uint32_t o[2][32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float a0, a1, a2, a3;
+        ld_shared_v4(sx + r * 128 + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
+        const uint32_t pk[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
+                                __float_as_uint(a3)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * c + e;                    // half2 index -> scores 2i, 2i+1
+          const float2 mine = unpack_half2(h[i]);
+          const float2 theirs = unpack_half2(pk[e]);
+          // both CTAs add the same two fp16-rounded halves: identical sums
+          o[(2 * i) >> 5][(2 * i) & 31] = __float_as_uint(mine.x + theirs.x);
+          o[(2 * i + 1) >> 5][(2 * i + 1) & 31] = __float_as_uint(mine.y + theirs.y);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(px_empty);
+      tmem_st32(tbase + lane_off + TM_S + slot * NT, o[0]);
+      tmem_st32(tbase + lane_off + TM_S + slot * NT + 32, o[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_comb[slot]);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- softmax (thread = head) + epilogue
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t sp_ = smem_u32(smem + OFF_P);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
       const int slot = j & 1;
-      if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
+      if (!warp_wait(&s_comb[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[2][32];
       tmem_ld32(tbase + lane_off + TM_S + slot * NT, sr[0]);
@@ -230,38 +297,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[slot]);
-      // exchange the partial scores with the peer CTA (row r, 16 chunks of 4,
-      // chunk position swizzled by the row to spread shared-memory banks)
-      if (!warp_wait_cluster(&x_empty, (j & 1) ^ 1, abort_v, p.status)) { ok = false; break; }
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int i = c >> 3, e = (c & 7) * 4;
-        st_async_v4(px + r * 256 + ((c ^ (r & 15)) << 4), sr[i][e], sr[i][e + 1], sr[i][e + 2],
-                    sr[i][e + 3], px_full);
-      }
-      if (r == 0) mbar_arrive_expect_tx(&x_full, 128 * NT * 4);
-      if (!warp_wait_cluster(&x_full, j & 1, abort_v, p.status)) { ok = false; break; }
-      float s[NT];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float a0, a1, a2, a3;
-        ld_shared_v4(sx + r * 256 + ((c ^ (r & 15)) << 4), a0, a1, a2, a3);
-        const int i = c >> 3, e = (c & 7) * 4;
-        s[c * 4 + 0] = __uint_as_float(sr[i][e + 0]) + a0;
-        s[c * 4 + 1] = __uint_as_float(sr[i][e + 1]) + a1;
-        s[c * 4 + 2] = __uint_as_float(sr[i][e + 2]) + a2;
-        s[c * 4 + 3] = __uint_as_float(sr[i][e + 3]) + a3;
-      }
-      mbar_arrive_remote(px_empty);
       // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
       const int lo = j * NT - (chunk_base(n, t0, j) - t0);
       const int hi = tcount - (chunk_base(n, t0, j) - t0);
-      float mx = m_ref;
+      float s[NT];
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
       for (int i = 0; i < NT; ++i) {
-        s[i] = (i >= lo && i < hi) ? s[i] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[i]);
+        const float v = __uint_as_float(sr[i >> 5][i & 31]) * p.scale_log2;
+        s[i] = (i >= lo && i < hi) ? v : -INFINITY;
+        mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
       }
+      const float mx = fmaxf(m_ref, fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))));
       const bool grow = mx > m_ref + kRescaleLog2;
       if (j > 0) {
         if (!warp_wait(&pv_done, (j - 1) & 1, abort_v, p.status)) { ok = false; break; }
@@ -284,7 +334,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         tmem_wait_st();
       }
-      float lsum = 0.f;
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t w[4];
@@ -292,12 +344,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int e = 0; e < 4; ++e) {
           const float p0 = ex2(s[ch * 8 + 2 * e] - m_ref);
           const float p1 = ex2(s[ch * 8 + 2 * e + 1] - m_ref);
-          lsum += p0 + p1;
+          ls[2 * e] += p0;
+          ls[2 * e + 1] += p1;
           w[e] = pack_bf16(p0, p1);
         }
         st_shared_v4(sp_ + r * 128 + ((ch ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
       }
-      l += lsum;
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
