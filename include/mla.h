@@ -290,6 +290,39 @@ MLA_API mla_status mla_check_device_status(void* workspace, void* stream);
 MLA_API mla_status mla_set_stage_events(void* const* events, int32_t n);
 MLA_API int64_t mla_kernel_launches(void);
 
+/*
+ * mla_decode_absorbed_noalloc -- mla_decode_absorbed for callers that cannot
+ * allocate device memory when they decode.  There is no counterpart in the
+ * pages; it exists for integration.  Typical callers: a host framework whose
+ * own pool owns every device allocation, a plugin that is only handed input
+ * and output tensors, a serving loop that forbids allocation on its latency
+ * path.  Instead of a caller workspace it uses one array of
+ * MLA_DECODE_NOALLOC_SCRATCH_BYTES that the library declares in device memory
+ * (every GPU that loads the library holds it until the process exits).
+ *
+ *   Arguments, layouts and results are those of mla_decode_absorbed without
+ *   the workspace pair.
+ *   Returns MLA_ERR_WORKSPACE (with mla_last_error_detail naming both sizes)
+ *   when mla_decode_workspace_size(cfg, B, max_ctx) exceeds the array, e.g.
+ *   B = 16 sequences of 128 heads up to max_ctx = 8192 fit; B = 64 does not.
+ *   The first call on each device looks up that device's copy of the array
+ *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.  The call allocates nothing: no cudaMalloc, cudaFree or
+ *   allocating library routine.
+ *   All calls on a device share the one array and leave the last call's
+ *   intermediates in it: calls whose work overlaps on the GPU (different
+ *   streams, or host threads racing) corrupt each other -- serialise them.
+ *   Device-side status (bounded-wait timeouts, out-of-range cu_ctx) is
+ *   recorded in the array but not reported; use mla_decode_absorbed with
+ *   mla_check_device_status where that report is needed.
+ */
+#define MLA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+MLA_API mla_status mla_decode_absorbed_noalloc(const mla_config* cfg, const void* q_nope,
+                                               const void* q_pe, const void* w_kv_b,
+                                               const void* latent_cache, const int32_t* cu_ctx,
+                                               int32_t B, int32_t max_ctx, const void* w_o,
+                                               void* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

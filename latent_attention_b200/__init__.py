@@ -15,7 +15,8 @@ from ._lib import (mla_config, mla_weights, mla_prefill_layout,
 __all__ = ["MlaError", "make_config", "mla_build_rope_tables",
            "mla_prefill_workspace_size", "mla_prefill_forward",
            "mla_decode_workspace_size", "mla_decode_absorbed",
-           "mla_check_device_status", "abi_version"]
+           "mla_check_device_status", "mla_decode_absorbed_noalloc",
+           "abi_version"]
 
 
 class MlaError(RuntimeError):
@@ -132,3 +133,16 @@ def mla_decode_absorbed(cfg, q_nope, q_pe, w_kv_b, latent_cache, cu_ctx, B,
 def mla_check_device_status(workspace, stream=None):
     _check(_lib.load().mla_check_device_status(_ptr(workspace, "workspace"),
                                                _stream(stream)))
+
+
+def mla_decode_absorbed_noalloc(cfg, q_nope, q_pe, w_kv_b, latent_cache, cu_ctx,
+                                B, max_ctx, w_o, out, stream=None):
+    """``mla_decode_absorbed`` for callers that cannot allocate device memory:
+    the library's own static device array replaces the workspace.  Calls on
+    one device share that array, so they must not overlap on the GPU."""
+    c = cfg if isinstance(cfg, mla_config) else make_config(cfg)
+    _check(_lib.load().mla_decode_absorbed_noalloc(
+        C.byref(c), _ptr(q_nope, "q_nope"), _ptr(q_pe, "q_pe"),
+        _ptr(w_kv_b, "w_kv_b"), _ptr(latent_cache, "latent_cache"),
+        _ptr(cu_ctx, "cu_ctx"), int(B), int(max_ctx), _ptr(w_o, "w_o", True),
+        _ptr(out, "out"), _stream(stream)))

@@ -16,6 +16,8 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_NULL", 2: "MLA_ERR_SHAPE",
                 6: "MLA_ERR_UNSUPPORTED", 7: "MLA_ERR_CUDA",
                 8: "MLA_ERR_DEVICE_TIMEOUT"}
 MLA_F32, MLA_BF16 = 0, 1
+# Size of the library's static decode scratch (mla.h MLA_DECODE_NOALLOC_SCRATCH_BYTES).
+DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ROPE_TYPES = {"none": 0, "plain": 1, "yarn": 2}
 
 # Every symbol the header declares (checked by the CPU tests).
@@ -23,7 +25,8 @@ EXPORTED = ["mla_abi_version", "mla_status_string", "mla_last_error_detail",
             "mla_build_rope_tables", "mla_prefill_workspace_size",
             "mla_prefill_forward", "mla_decode_workspace_size",
             "mla_decode_absorbed", "mla_check_device_status",
-            "mla_set_stage_events", "mla_kernel_launches"]
+            "mla_set_stage_events", "mla_kernel_launches",
+            "mla_decode_absorbed_noalloc"]
 
 
 class mla_config(C.Structure):
@@ -99,5 +102,8 @@ def load():
     lib.mla_set_stage_events.argtypes = [C.POINTER(vp), i32]
     lib.mla_kernel_launches.restype = C.c_int64
     lib.mla_kernel_launches.argtypes = []
+    lib.mla_decode_absorbed_noalloc.restype = C.c_int
+    lib.mla_decode_absorbed_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, i32, vp,
+                                                vp, vp]
     _lib = lib
     return lib

@@ -139,6 +139,7 @@ char* at(void* ws, int64_t off) { return off < 0 ? nullptr : static_cast<char*>(
 }  // namespace
 
 namespace mla {
+void set_error_detail(const char* msg) { g_detail = msg; }
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 void stage_event(int i, cudaStream_t st) {
   if (i < g_n_events && g_events[i]) cudaEventRecord(g_events[i], st);

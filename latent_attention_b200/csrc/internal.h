@@ -107,6 +107,8 @@ struct DecodeArgs {
 
 // Launch accounting and stage events (defined in api.cu).
 void count_launches(int n = 1);
+// Sets the text mla_last_error_detail() returns on this host thread.
+void set_error_detail(const char* msg);
 // Records registered stage event i (if any) on stream st.
 void stage_event(int i, cudaStream_t st);
 
