@@ -17,12 +17,13 @@
 //   warp 0     TMA: Q (once) and the K ring (2 stages of 3 boxes)
 //   warp 1     TMEM allocation and MMA issue: S_j = Q K_j^T (12 x M128 N128
 //              K16) into one of two TMEM S buffers, then O += P_{j-1} V_{j-1}
-//   warp 2     TMA: V (single stage, 2 boxes of 64 value columns)
+//   warp 2     TMA: V (2 stages, 2 boxes of 64 value columns)
 //   warps 4-7  softmax, thread = query row: S row from TMEM, mask, running
 //              max with lazy rescaling (O and l rescaled only when the max
-//              grows by more than 2^8), P as bf16 into shared memory in the
-//              128-byte swizzled K-major layout, final O / l to global.
-// TMEM: S0 [0,128), S1 [128,256), O [256,384).  All waits are bounded.
+//              grows by more than 2^8), P as bf16 into TMEM (the A operand of
+//              the PV MMA is read from tensor memory), final O / l to global.
+// TMEM: S0 [0,128), S1 [128,256), O [256,384), P [384,448).  All waits are
+// bounded.
 #include "sm100.cuh"
 #include "tc.h"
 
@@ -36,14 +37,13 @@ constexpr int DN = 128, DR = 64, DV = 128, DQ = DN + DR;
 constexpr int BOX = 128 * 64 * 2;                // one 64-column box of 128 rows
 constexpr int Q_BYTES = 3 * BOX;                 // 48 KB
 constexpr int K_BYTES = 3 * BOX;                 // 48 KB per stage
-constexpr int V_BYTES = 2 * BOX;                 // 32 KB
-constexpr int P_BYTES = 2 * BOX;                 // 32 KB
-constexpr int OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + 2 * K_BYTES, OFF_P = OFF_V + V_BYTES;
-constexpr int SMEM_BYTES = OFF_P + P_BYTES + 1024;
+constexpr int V_BYTES = 2 * BOX;                 // 32 KB per stage
+constexpr int OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + 2 * K_BYTES;
+constexpr int SMEM_BYTES = OFF_V + 2 * V_BYTES + 1024;
 constexpr int NTHREADS = 256;
 constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, DV, 0, 1);   // V is MN-major
-constexpr uint32_t TM_S = 0, TM_O = 256;
+constexpr uint32_t TM_S = 0, TM_O = 256, TM_P = 384;   // P: 2 slots of 64 columns
 constexpr float kRescaleLog2 = 8.f;
 
 struct AttnTcParams {
@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmKpe,
                    const __grid_constant__ AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, k_full[2], k_empty[2], v_full, v_empty, s_full[2],
-      s_free[2], p_full, pv_done;
+  __shared__ __align__(8) uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2],
+      s_full[2], s_free[2], p_full, pv_done[2];
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -69,9 +69,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_v = &abort_flag;
 
-  const int hh = blockIdx.x % p.h;
-  const int b = blockIdx.x / p.h;
-  const int qb = p.n_qblk - 1 - blockIdx.y;         // heavy blocks first
+  // All query blocks of one head run together (heaviest first), so that the
+  // head's keys and values come from HBM once and from L2 for the others.
+  const int hh = blockIdx.y % p.h;
+  const int b = blockIdx.y / p.h;
+  const int qb = p.n_qblk - 1 - blockIdx.x;
   const int q0 = qb * BQ;
   const int row0 = b * p.T;                          // first token of the sequence
   const int nkv = qb + 1;                            // causal: key blocks 0..qb
@@ -83,11 +85,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&k_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 4);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
-    mbar_init(&v_full, 1);
-    mbar_init(&v_empty, 1);
     mbar_init(&p_full, 4);
-    mbar_init(&pv_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -124,33 +127,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ---------------- V producer
     if (elect_one()) {
       for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&v_empty, (j & 1) ^ 1, abort_v, p.status)) break;
-        uint8_t* sv = smem + OFF_V;
-        mbar_arrive_expect_tx(&v_full, V_BYTES);
+        const int slot = j & 1;
+        if (!mbar_wait(&v_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
+        uint8_t* sv = smem + OFF_V + slot * V_BYTES;
+        mbar_arrive_expect_tx(&v_full[slot], V_BYTES);
         const int kr = row0 + j * BKV;
-        tma_load_2d(sv, &tmKV, hh * (DN + DV) + DN, kr, &v_full);
-        tma_load_2d(sv + BOX, &tmKV, hh * (DN + DV) + DN + 64, kr, &v_full);
+        tma_load_2d(sv, &tmKV, hh * (DN + DV) + DN, kr, &v_full[slot]);
+        tma_load_2d(sv + BOX, &tmKV, hh * (DN + DV) + DN + 64, kr, &v_full[slot]);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (elect_one()) {
       const uint32_t sq = smem_u32(smem + OFF_Q);
-      const uint32_t sp = smem_u32(smem + OFF_P);
-      const uint32_t sv = smem_u32(smem + OFF_V);
       bool ok = mbar_wait(&q_full, 0, abort_v, p.status);
       auto issue_pv = [&](int j) -> bool {
+        const int vs = j & 1;
         if (!mbar_wait(&p_full, j & 1, abort_v, p.status)) return false;
-        if (!mbar_wait(&v_full, j & 1, abort_v, p.status)) return false;
+        if (!mbar_wait(&v_full[vs], (j >> 1) & 1, abort_v, p.status)) return false;
         tc_fence_after();
+        const uint32_t sv = smem_u32(smem + OFF_V + vs * V_BYTES);
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k) {
-          const uint64_t a = desc_kmajor_sw128(sp + (k >> 2) * BOX + (k & 3) * 32);
+          // A = P_j from TMEM slot j % 2: 16 keys = 8 packed columns per step
           const uint64_t bv = desc_mnmajor_sw128(sv + k * 16 * 128, BOX);
-          mma_bf16(tbase + TM_O, a, bv, IDESC_PV, (j | k) != 0);
+          mma_bf16_ts(tbase + TM_O, tbase + TM_P + (j & 1) * 64 + k * 8, bv, IDESC_PV,
+                      (j | k) != 0);
         }
-        mma_commit(&v_empty);
-        mma_commit(&pv_done);
+        mma_commit(&v_empty[vs]);
+        mma_commit(&pv_done[j & 1]);
         return true;
       };
       for (int j = 0; ok && j < nkv; ++j) {
@@ -180,7 +185,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int r = quad * 32 + lane;                  // query row within the block
     const int qi = q0 + r;                           // query position
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t sp = smem_u32(smem + OFF_P);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
@@ -195,32 +199,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[slot]);
 
+      // Raw scores; the scale is folded into the exp argument below (scale > 0,
+      // so the row max commutes with it).  The causal compare is needed only on
+      // the diagonal block and on the ragged tail.
       float s[128];
       const int k0 = j * BKV;
       const int kmax = min(qi, p.T - 1) - k0;         // last visible key in this block
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kk = c * 32 + i;
-          const float v = __uint_as_float(sr[c][i]) * p.scale_log2;
-          s[kk] = kk <= kmax ? v : -INFINITY;
-        }
-      float mx = m_ref;
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
+      if (kmax < 127) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) mx = fmaxf(mx, s[i]);
-      const bool grow = mx > m_ref + kRescaleLog2;    // also true for the first block
-      if (j > 0) {
-        if (!warp_wait(&pv_done, (j - 1) & 1, abort_v, p.status)) { ok = false; break; }
-        tc_fence_after();
+        for (int i = 0; i < 128; ++i)
+          if (i > kmax) s[i] = -INFINITY;
       }
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      const float mx = fmaxf(m_ref, p.scale_log2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]),
+                                                                fmaxf(mx8[2], mx8[3])),
+                                                          fmaxf(fmaxf(mx8[4], mx8[5]),
+                                                                fmaxf(mx8[6], mx8[7]))));
+      const bool grow = mx > m_ref + kRescaleLog2;    // also true for the first block
       const float alpha = grow ? ex2(m_ref - mx) : 1.f;
       if (grow) {
         l *= alpha;
         m_ref = mx;
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // rescale this row's O accumulator (warp-collective TMEM access)
+      // P = 2^(scale * s - m_ref) as packed bf16 pairs (computed before any wait)
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+      const float sc = p.scale_log2;
+      uint32_t w[2][32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int i = half * 64 + 2 * e;
+          const float p0 = ex2(fmaf(s[i], sc, -m_ref));
+          const float p1 = ex2(fmaf(s[i + 1], sc, -m_ref));
+          ls[e & 7] += p0 + p1;
+          w[half][e] = pack_bf16(p0, p1);
+        }
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      // A rescale of O needs every earlier PV finished (PV_{j-1} is the last);
+      // otherwise only the PV that read this P slot two blocks ago must be done.
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
+      if (rescale) {
+        if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
@@ -230,31 +264,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tbase + lane_off + TM_O + c * 32, o);
         }
-        tmem_wait_st();
-      }
-      // P = 2^(s - m_ref) as bf16, swizzled K-major rows of the A operand.
-      float lsum = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(s[ch * 8 + 2 * e] - m_ref);
-          const float p1 = ex2(s[ch * 8 + 2 * e + 1] - m_ref);
-          lsum += p0 + p1;
-          w[e] = pack_bf16(p0, p1);
+      } else if (j > 1) {
+        if (!warp_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
         }
-        const int atom = ch >> 3, c16 = ch & 7;
-        const uint32_t addr = sp + atom * BOX + r * 128 + ((c16 ^ (r & 7)) << 4);
-        st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+        tc_fence_after();
       }
-      l += lsum;
-      fence_proxy_async();
+      tmem_st32(tbase + lane_off + TM_P + (j & 1) * 64, w[0]);
+      tmem_st32(tbase + lane_off + TM_P + (j & 1) * 64 + 32, w[1]);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full);
     }
-    if (ok && warp_wait(&pv_done, (nkv - 1) & 1, abort_v, p.status)) {
+    if (ok && warp_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = qi < p.T;
@@ -328,7 +352,7 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(a.h * a.B, p.n_qblk);
+  dim3 grid(p.n_qblk, a.h * a.B);
   attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmKV, tmKpe, p);
   count_launches();
   return cudaGetLastError();
