@@ -28,7 +28,8 @@
 // without further exchange.  Warp roles (256 threads per CTA):
 //   warp 0     TMA: Q share once, chunk ring (2 stages), L2 prefetch ahead
 //   warp 1     TMEM allocation, MMA issue (S_j, then O += P_{j-1} C_{j-1})
-//   warps 4-7  score exchange + softmax (thread = head) + epilogue
+//   warps 2, 3, 8, 9  score exchange, one chunk ahead of the softmax
+//   warps 4-7  softmax (thread = head), P into TMEM, epilogue
 // All waits are bounded; a timeout sets the device status word.
 #include <cfloat>
 #include <cuda_fp16.h>
@@ -49,14 +50,16 @@ constexpr int MAX_ATOMS = 5;
 constexpr int OFF_Q = 0;
 constexpr int OFF_C = OFF_Q + MAX_ATOMS * QBOX;          // 80 KB
 constexpr int STAGE = MAX_ATOMS * CBOX;                  // 40 KB
-constexpr int OFF_X = OFF_C + 2 * STAGE;                 // exchange: 128 x 64 fp16
-constexpr int OFF_P = OFF_X + 128 * NT * 2;              // P: 128 x 64 bf16
-constexpr int SMEM_BYTES = OFF_P + 128 * NT * 2 + 1024;
+constexpr int XBUF = 128 * NT * 2;                       // exchange: 128 x 64 fp16
+constexpr int OFF_X = OFF_C + 2 * STAGE;                 // two exchange buffers
+constexpr int SMEM_BYTES = OFF_X + 2 * XBUF + 1024;
 constexpr int NTHREADS = 320;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
-constexpr uint32_t TM_S = 0, TM_O = 256;
+// TMEM: S slots [0, 128), P slots (128 rows x 64 keys bf16 = 32 columns each)
+// [128, 192), O [256, 512).
+constexpr uint32_t TM_S = 0, TM_P = 128, TM_O = 256;
 constexpr float kRescaleLog2 = 8.f;
 
 struct DecTcParams {
@@ -109,7 +112,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full, c_full[2], c_empty[2], s_full[2], s_comb[2],
-      s_free[2], p_full, pv_done, x_full, x_empty;
+      s_free[2], p_full, pv_done[2], x_full[2], x_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -145,9 +148,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_init(&s_free[s], 4);
     }
     mbar_init(&p_full, 4);
-    mbar_init(&pv_done, 1);
-    mbar_init(&x_full, 1);     // one local arrive.expect_tx + the peer's st.async bytes
-    mbar_init(&x_empty, 4);    // one arrive per exchange warp of the peer
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&x_full[s], 1);    // one local arrive.expect_tx + the peer's st.async bytes
+      mbar_init(&x_empty[s], 4);   // one arrive per exchange warp of the peer
+    }
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -192,18 +198,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     if (elect_one()) {
       const uint32_t sq = smem_u32(smem + OFF_Q);
-      const uint32_t sp_ = smem_u32(smem + OFF_P);
       bool ok = mbar_wait(&q_full, 0, abort_v, p.status);
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait(&p_full, j & 1, abort_v, p.status)) return false;
         tc_fence_after();
         const uint32_t sc = smem_u32(smem + OFF_C + (j & 1) * STAGE);
 #pragma unroll
-        for (int k = 0; k < NT / 16; ++k)
-          mma_bf16(tbase + TM_O, desc_kmajor_sw128(sp_ + k * 32),
-                   desc_mnmajor_sw128(sc + k * 16 * 128, CBOX), IDESC_PV, (j | k) != 0);
+        for (int k = 0; k < NT / 16; ++k)   // A = P_j from TMEM slot j % 2, 8 columns per step
+          mma_bf16_ts(tbase + TM_O, tbase + TM_P + (j & 1) * 32 + k * 8,
+                      desc_mnmajor_sw128(sc + k * 16 * 128, CBOX), IDESC_PV, (j | k) != 0);
         mma_commit(&c_empty[j & 1]);
-        mma_commit(&pv_done);
+        mma_commit(&pv_done[j & 1]);
         return true;
       };
       for (int j = 0; ok && j < nch; ++j) {
@@ -228,12 +233,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t sx = smem_u32(smem + OFF_X);
-    const uint32_t px = map_peer(sx, peer);
-    const uint32_t px_full = map_peer(smem_u32(&x_full), peer);
-    const uint32_t px_empty = map_peer(smem_u32(&x_empty), peer);
     for (int j = 0; j < nch; ++j) {
       const int slot = j & 1;
+      // exchange buffer j % 2: the peer's send of chunk j only needs this
+      // CTA to have consumed chunk j - 2 from the same buffer
+      const uint32_t sx = smem_u32(smem + OFF_X + slot * XBUF);
+      const uint32_t px = map_peer(sx, peer);
+      const uint32_t px_full = map_peer(smem_u32(&x_full[slot]), peer);
+      const uint32_t px_empty = map_peer(smem_u32(&x_empty[slot]), peer);
       if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) break;
       tc_fence_after();
       uint32_t sr[2][32];
@@ -245,13 +252,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (int i = 0; i < 32; ++i)
         h[i] = pack_half2(__uint_as_float(sr[i >> 4][(2 * i) & 31]),
                           __uint_as_float(sr[i >> 4][(2 * i + 1) & 31]));
-      if (!warp_wait_cluster(&x_empty, (j & 1) ^ 1, abort_v, p.status)) break;
+      if (!warp_wait_cluster(&x_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         st_async_v4(px + r * 128 + ((c ^ (r & 7)) << 4), h[4 * c], h[4 * c + 1], h[4 * c + 2],
                     h[4 * c + 3], px_full);
-      if (r == 0) mbar_arrive_expect_tx(&x_full, 128 * NT * 2);
-      if (!warp_wait_cluster(&x_full, j & 1, abort_v, p.status)) break;
+      if (r == 0) mbar_arrive_expect_tx(&x_full[slot], XBUF);
+      if (!warp_wait_cluster(&x_full[slot], (j >> 1) & 1, abort_v, p.status)) break;
       uint32_t o[2][32];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -283,7 +290,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t sp_ = smem_u32(smem + OFF_P);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
@@ -313,16 +319,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const float mx = fmaxf(m_ref, fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))));
       const bool grow = mx > m_ref + kRescaleLog2;
-      if (j > 0) {
-        if (!warp_wait(&pv_done, (j - 1) & 1, abort_v, p.status)) { ok = false; break; }
-        tc_fence_after();
-      }
       const float alpha = grow ? ex2(m_ref - mx) : 1.f;
       if (grow) {
         l *= alpha;
         m_ref = mx;
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+      uint32_t w[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = ex2(s[2 * e] - m_ref);
+        const float p1 = ex2(s[2 * e + 1] - m_ref);
+        ls[e & 7] += p0 + p1;
+        w[e] = pack_bf16(p0, p1);
+      }
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      // A rescale of O needs every earlier PV finished (PV_{j-1} is the last);
+      // otherwise only the PV that read this P slot two chunks ago must be done.
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
+      if (rescale) {
+        if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
@@ -332,31 +354,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tbase + lane_off + TM_O + c * 32, o);
         }
-        tmem_wait_st();
-      }
-      float ls[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(s[ch * 8 + 2 * e] - m_ref);
-          const float p1 = ex2(s[ch * 8 + 2 * e + 1] - m_ref);
-          ls[2 * e] += p0;
-          ls[2 * e + 1] += p1;
-          w[e] = pack_bf16(p0, p1);
+      } else if (j > 1) {
+        if (!warp_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
         }
-        st_shared_v4(sp_ + r * 128 + ((ch ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+        tc_fence_after();
       }
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      fence_proxy_async();
+      tmem_st32(tbase + lane_off + TM_P + (j & 1) * 32, w);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full);
     }
-    if (ok && warp_wait(&pv_done, (nch - 1) & 1, abort_v, p.status)) {
+    if (ok && warp_wait(&pv_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const int head = h0 + r;
       const bool head_ok = head < p.h;
