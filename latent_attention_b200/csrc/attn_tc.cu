@@ -12,18 +12,25 @@
 // head dim and no trimming (the FA2 constraint the verl kimi_vl page works
 // around does not apply).
 //
-// One CTA = (batch, head, 128-query block); heaviest causal blocks launch
-// first.  Warp roles (256 threads):
-//   warp 0     TMA: Q (once) and the K ring (2 stages of 3 boxes)
-//   warp 1     TMEM allocation and MMA issue: S_j = Q K_j^T (12 x M128 N128
-//              K16) into one of two TMEM S buffers, then O += P_{j-1} V_{j-1}
-//   warp 2     TMA: V (2 stages, 2 boxes of 64 value columns)
-//   warps 4-7  softmax, thread = query row: S row from TMEM, mask, running
-//              max with lazy rescaling (O and l rescaled only when the max
-//              grows by more than 2^8), P as bf16 into TMEM (the A operand of
-//              the PV MMA is read from tensor memory), final O / l to global.
-// TMEM: S0 [0,128), S1 [128,256), O [256,384), P [384,448).  All waits are
-// bounded.
+// One CTA = (batch, head, two 128-query tiles A and B); every K/V block it
+// loads serves both tiles.  All query tiles of one head run together
+// (heaviest first), so a head's keys and values leave HBM once.  Warp roles
+// (384 threads):
+//   warp 0       TMA: Q of both tiles (once), K (one stage of 3 boxes)
+//   warp 2       TMA: V ring (2 stages of 2 boxes of 64 value columns)
+//   warp 1       TMEM allocation and MMA issue, in the order
+//                  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
+//                so that the tensor core works on one tile while the other
+//                tile's softmax runs; S_X(j+1) is issued once PV_X(j) has
+//                completed (P_X(j) lives in S_X's columns).
+//   warps 4-7    softmax of tile A, warps 8-11 softmax of tile B (thread =
+//                query row): S from TMEM, causal mask on the diagonal block,
+//                running max with lazy rescaling (O and l rescaled only when
+//                the max grows by more than 2^8), P as bf16 pairs written
+//                over the first 64 columns of S (the A operand of PV, read
+//                from tensor memory), final O / l to global.
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).  Every wait
+// is bounded.
 #include "sm100.cuh"
 #include "tc.h"
 
@@ -35,21 +42,21 @@ using namespace sm100;
 constexpr int BQ = 128, BKV = 128;
 constexpr int DN = 128, DR = 64, DV = 128, DQ = DN + DR;
 constexpr int BOX = 128 * 64 * 2;                // one 64-column box of 128 rows
-constexpr int Q_BYTES = 3 * BOX;                 // 48 KB
+constexpr int Q_BYTES = 3 * BOX;                 // 48 KB per tile
 constexpr int K_BYTES = 3 * BOX;                 // 48 KB per stage
-constexpr int V_BYTES = 2 * BOX;                 // 32 KB per stage
-constexpr int OFF_Q = 0, OFF_K = Q_BYTES, OFF_V = OFF_K + 2 * K_BYTES;
+constexpr int V_BYTES = 2 * BOX;                 // 32 KB
+constexpr int OFF_Q = 0, OFF_K = 2 * Q_BYTES, OFF_V = OFF_K + K_BYTES;
 constexpr int SMEM_BYTES = OFF_V + 2 * V_BYTES + 1024;
-constexpr int NTHREADS = 256;
+constexpr int NTHREADS = 384;
 constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, DV, 0, 1);   // V is MN-major
-constexpr uint32_t TM_S = 0, TM_O = 256, TM_P = 384;   // P: 2 slots of 64 columns
+constexpr uint32_t TM_S = 0, TM_O = 256;                   // + 128 * tile
 constexpr float kRescaleLog2 = 8.f;
 
 struct AttnTcParams {
   int B, T, h;
   float scale_log2;      // softmax scale * log2(e)
-  int n_qblk;
+  int n_pairs;           // CTAs per head: ceil(T / 256)
   __nv_bfloat16* o;      // [N, h, DV]
   uint32_t* status;
 };
@@ -60,8 +67,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmKpe,
                    const __grid_constant__ AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2],
-      s_full[2], s_free[2], p_full, pv_done[2];
+  __shared__ __align__(8) uint64_t q_full, k_full, k_empty, v_full[2], v_empty[2], s_full[2],
+      p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -69,28 +76,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_v = &abort_flag;
 
-  // All query blocks of one head run together (heaviest first), so that the
-  // head's keys and values come from HBM once and from L2 for the others.
   const int hh = blockIdx.y % p.h;
   const int b = blockIdx.y / p.h;
-  const int qb = p.n_qblk - 1 - blockIdx.x;
-  const int q0 = qb * BQ;
+  const int c = p.n_pairs - 1 - blockIdx.x;          // heaviest pair first
   const int row0 = b * p.T;                          // first token of the sequence
-  const int nkv = qb + 1;                            // causal: key blocks 0..qb
+  // tile X covers queries [q0X, q0X + 128) and key blocks [0, nkvX)
+  const int q0A = 256 * c, q0B = 256 * c + BQ;
+  const int nkvA = q0A < p.T ? min(q0A + BQ - 1, p.T - 1) / BKV + 1 : 0;
+  const int nkvB = q0B < p.T ? min(q0B + BQ - 1, p.T - 1) / BKV + 1 : 0;
+  const int nkv = max(nkvA, nkvB);
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 4);
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 4);
+      mbar_init(&pv_done[s], 1);
     }
-    mbar_init(&p_full, 4);
-    mbar_init(&pv_done[0], 1);
-    mbar_init(&pv_done[1], 1);
+    mbar_init(&k_full, 1);
+    mbar_init(&k_empty, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -108,19 +114,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tma_prefetch(&tmQ);
       tma_prefetch(&tmKV);
       tma_prefetch(&tmKpe);
-      uint8_t* sq = smem + OFF_Q;
-      mbar_arrive_expect_tx(&q_full, Q_BYTES);
-      for (int a = 0; a < 3; ++a)
-        tma_load_2d(sq + a * BOX, &tmQ, hh * DQ + a * 64, row0 + q0, &q_full);
+      mbar_arrive_expect_tx(&q_full, (nkvB > 0 ? 2 : 1) * Q_BYTES);
+      for (int a = 0; a < 3; ++a) {
+        tma_load_2d(smem + OFF_Q + a * BOX, &tmQ, hh * DQ + a * 64, row0 + q0A, &q_full);
+        if (nkvB > 0)
+          tma_load_2d(smem + OFF_Q + Q_BYTES + a * BOX, &tmQ, hh * DQ + a * 64, row0 + q0B,
+                      &q_full);
+      }
       for (int j = 0; j < nkv; ++j) {
-        const int slot = j & 1;
-        if (!mbar_wait(&k_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
-        uint8_t* sk = smem + OFF_K + slot * K_BYTES;
-        mbar_arrive_expect_tx(&k_full[slot], K_BYTES);
+        if (!mbar_wait(&k_empty, (j & 1) ^ 1, abort_v, p.status)) break;
+        uint8_t* sk = smem + OFF_K;
+        mbar_arrive_expect_tx(&k_full, K_BYTES);
         const int kr = row0 + j * BKV;
-        tma_load_2d(sk, &tmKV, hh * (DN + DV), kr, &k_full[slot]);
-        tma_load_2d(sk + BOX, &tmKV, hh * (DN + DV) + 64, kr, &k_full[slot]);
-        tma_load_2d(sk + 2 * BOX, &tmKpe, 0, kr, &k_full[slot]);
+        tma_load_2d(sk, &tmKV, hh * (DN + DV), kr, &k_full);
+        tma_load_2d(sk + BOX, &tmKV, hh * (DN + DV) + 64, kr, &k_full);
+        tma_load_2d(sk + 2 * BOX, &tmKpe, 0, kr, &k_full);
       }
     }
   } else if (warp == 2) {
@@ -140,85 +148,98 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ---------------- MMA issuer
     if (elect_one()) {
       const uint32_t sq = smem_u32(smem + OFF_Q);
-      bool ok = mbar_wait(&q_full, 0, abort_v, p.status);
-      auto issue_pv = [&](int j) -> bool {
-        const int vs = j & 1;
-        if (!mbar_wait(&p_full, j & 1, abort_v, p.status)) return false;
-        if (!mbar_wait(&v_full[vs], (j >> 1) & 1, abort_v, p.status)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(smem + OFF_V + vs * V_BYTES);
-#pragma unroll
-        for (int k = 0; k < BKV / 16; ++k) {
-          // A = P_j from TMEM slot j % 2: 16 keys = 8 packed columns per step
-          const uint64_t bv = desc_mnmajor_sw128(sv + k * 16 * 128, BOX);
-          mma_bf16_ts(tbase + TM_O, tbase + TM_P + (j & 1) * 64 + k * 8, bv, IDESC_PV,
-                      (j | k) != 0);
-        }
-        mma_commit(&v_empty[vs]);
-        mma_commit(&pv_done[j & 1]);
-        return true;
-      };
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int slot = j & 1;
-        if (!mbar_wait(&k_full[slot], (j >> 1) & 1, abort_v, p.status)) break;
-        if (!mbar_wait(&s_free[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + OFF_K + slot * K_BYTES);
+      const int nkvX[2] = {nkvA, nkvB};
+      // S_X(j) = Q_X K_j^T into TMEM S_X (K_j in the single K stage)
+      auto issue_s = [&](int x, int j) {
+        const uint32_t sk = smem_u32(smem + OFF_K);
+        const uint32_t qx = sq + x * Q_BYTES;
 #pragma unroll
         for (int k = 0; k < DQ / 16; ++k) {
           const uint32_t off = (k >> 2) * BOX + (k & 3) * 32;
-          mma_bf16(tbase + TM_S + slot * BKV, desc_kmajor_sw128(sq + off),
+          mma_bf16(tbase + TM_S + x * 128, desc_kmajor_sw128(qx + off),
                    desc_kmajor_sw128(sk + off), IDESC_S, k != 0);
         }
-        mma_commit(&k_empty[slot]);
-        mma_commit(&s_full[slot]);
-        if (j > 0 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
-        }
+        mma_commit(&s_full[x]);
+      };
+      // O_X += P_X(j) V_j, P_X(j) from TMEM (16 keys = 8 packed columns per step)
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t sv = smem_u32(smem + OFF_V + (j & 1) * V_BYTES);
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k)
+          mma_bf16_ts(tbase + TM_O + x * 128, tbase + TM_S + x * 128 + k * 8,
+                      desc_mnmajor_sw128(sv + k * 16 * 128, BOX), IDESC_PV, (j | k) != 0);
+        mma_commit(&pv_done[x]);
+      };
+      bool ok = mbar_wait(&q_full, 0, abort_v, p.status) &&
+                mbar_wait(&k_full, 0, abort_v, p.status);
+      if (ok) {
+        tc_fence_after();
+        for (int x = 0; x < 2; ++x)
+          if (nkvX[x] > 0) issue_s(x, 0);
+        mma_commit(&k_empty);
       }
-      if (ok) issue_pv(nkv - 1);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const bool more = j + 1 < nkv;
+        bool k_ready = false;
+        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_v, p.status)) break;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (j < nkvX[x]) {
+            if (!mbar_wait(&p_full[x], j & 1, abort_v, p.status)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(x, j);
+          }
+          if (j + 1 < nkvX[x]) {
+            if (!k_ready) {       // K_{j+1} is waited for only where it is needed
+              if (!mbar_wait(&k_full, (j + 1) & 1, abort_v, p.status)) { ok = false; break; }
+              k_ready = true;
+            }
+            // S_X(j+1) overwrites the columns P_X(j) occupies: wait for PV_X(j)
+            if (!mbar_wait(&pv_done[x], j & 1, abort_v, p.status)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(x, j + 1);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&v_empty[j & 1]);
+        if (more) mma_commit(&k_empty);
+      }
     }
   } else if (warp >= 4) {
-    // ---------------- softmax warpgroup
+    // ---------------- softmax warpgroups: warps 4-7 tile A, 8-11 tile B
+    const int x = warp >= 8 ? 1 : 0;
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;                  // query row within the block
-    const int qi = q0 + r;                           // query position
+    const int r = quad * 32 + lane;                  // query row within the tile
+    const int qi = (x ? q0B : q0A) + r;              // query position
+    const int my_nkv = x ? nkvB : nkvA;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tbase + lane_off + TM_S + x * 128;
+    const uint32_t tO = tbase + lane_off + TM_O + x * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int slot = j & 1;
-      if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
+    for (int j = 0; j < my_nkv; ++j) {
+      // S_X(j) completion also implies PV_X(j-1) completion (in-order MMAs,
+      // and S_X(j) was issued after PV_X(j-1) completed)
+      if (!warp_wait(&s_full[x], j & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + lane_off + TM_S + slot * BKV + c * 32, sr[c]);
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, sr[cc]);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[slot]);
-
-      // Raw scores; the scale is folded into the exp argument below (scale > 0,
-      // so the row max commutes with it).  The causal compare is needed only on
-      // the diagonal block and on the ragged tail.
-      float s[128];
-      const int k0 = j * BKV;
-      const int kmax = min(qi, p.T - 1) - k0;         // last visible key in this block
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
+      // Raw scores; the scale is folded into the exp argument below (scale > 0).
+      const int kmax = min(qi, p.T - 1) - j * BKV;   // last visible key in this block
       if (kmax < 127) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > kmax) s[i] = -INFINITY;
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (cc * 32 + i > kmax) sr[cc][i] = __float_as_uint(-INFINITY);
       }
       float mx8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+      for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      for (int i = 8; i < 128; ++i)
+        mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[i >> 5][i & 31]));
       const float mx = fmaxf(m_ref, p.scale_log2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]),
                                                                 fmaxf(mx8[2], mx8[3])),
                                                           fmaxf(fmaxf(mx8[4], mx8[5]),
@@ -229,69 +250,57 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         l *= alpha;
         m_ref = mx;
       }
-      // P = 2^(scale * s - m_ref) as packed bf16 pairs (computed before any wait)
+      // P = 2^(scale * s - m_ref) as bf16 pairs over S's first 64 columns
       float ls[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
       const float sc = p.scale_log2;
-      uint32_t w[2][32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half)
+      for (int half = 0; half < 2; ++half) {
+        uint32_t w[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int i = half * 64 + 2 * e;
-          const float p0 = ex2(fmaf(s[i], sc, -m_ref));
-          const float p1 = ex2(fmaf(s[i + 1], sc, -m_ref));
+          const float p0 = ex2(fmaf(__uint_as_float(sr[i >> 5][i & 31]), sc, -m_ref));
+          const float p1 =
+              ex2(fmaf(__uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]), sc, -m_ref));
           ls[e & 7] += p0 + p1;
-          w[half][e] = pack_bf16(p0, p1);
+          w[e] = pack_bf16(p0, p1);
         }
+        tmem_st32(tS + half * 32, w);
+      }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      // A rescale of O needs every earlier PV finished (PV_{j-1} is the last);
-      // otherwise only the PV that read this P slot two blocks ago must be done.
-      const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
-      if (rescale) {
-        if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_X holds the sum through block j-1 (complete, see above)
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tbase + lane_off + TM_O + c * 32, o);
+          tmem_ld32(tO + cc * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tbase + lane_off + TM_O + c * 32, o);
+          tmem_st32(tO + cc * 32, o);
         }
-      } else if (j > 1) {
-        if (!warp_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
       }
-      tmem_st32(tbase + lane_off + TM_P + (j & 1) * 64, w[0]);
-      tmem_st32(tbase + lane_off + TM_P + (j & 1) * 64 + 32, w[1]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full);
+      if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    if (ok && warp_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_v, p.status)) {
+    if (ok && my_nkv > 0 && warp_wait(&pv_done[x], (my_nkv - 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = qi < p.T;
       __nv_bfloat16* dst = p.o + ((int64_t)(row0 + qi) * p.h + hh) * DV;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        tmem_ld32(tbase + lane_off + TM_O + c * 32, o);
+        tmem_ld32(tO + cc * 32, o);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8)
-            st_global_v4(dst + c * 32 + i,
+            st_global_v4(dst + cc * 32 + i,
                          pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv),
                          pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv),
                          pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv),
@@ -342,7 +351,7 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
   p.T = a.T;
   p.h = a.h;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.n_qblk = (a.T + BQ - 1) / BQ;
+  p.n_pairs = (a.T + 2 * BQ - 1) / (2 * BQ);
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
   p.status = a.status;
   static bool attr = false;
@@ -352,7 +361,7 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(p.n_qblk, a.h * a.B);
+  dim3 grid(p.n_pairs, a.h * a.B);
   attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmKV, tmKpe, p);
   count_launches();
   return cudaGetLastError();
