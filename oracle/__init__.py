@@ -20,12 +20,15 @@ Functions and what pins them (tests/test_oracle_pins.py):
   T=1 and equal-key special cases.
 * ``decode_absorbed`` / ``decode_unabsorbed`` -- agree with each other and
   with the last row of a prefill.
+* ``prefill_chunked`` -- equals the last rows of a full prefill whose first
+  positions produced the cache; reduces to ``prefill`` with no history.
 """
 from .mla_oracle import (yarn_get_mscale, softmax_scale, rope_frequencies,
                          rope_tables, rms_norm, rotate_half, apply_rope,
-                         prefill, decode_absorbed, decode_unabsorbed,
-                         max_rel_err)
+                         prefill, prefill_chunked, decode_absorbed,
+                         decode_unabsorbed, max_rel_err)
 
 __all__ = ["yarn_get_mscale", "softmax_scale", "rope_frequencies",
            "rope_tables", "rms_norm", "rotate_half", "apply_rope", "prefill",
+           "prefill_chunked",
            "decode_absorbed", "decode_unabsorbed", "max_rel_err"]

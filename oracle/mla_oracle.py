@@ -264,6 +264,73 @@ def prefill(cfg, inp, rows: Optional[Sequence[int]] = None,
 
 
 # ---------------------------------------------------------------------------
+# Chunked prefill against a cached latent
+# ---------------------------------------------------------------------------
+def prefill_chunked(cfg, inp, past_cache, T_past: int,
+                    return_parts: bool = False):
+    """T_new new tokens per sequence after T_past cached ones.
+
+    [MEGATRON] 推理优化: with cache_mla_latents the cache holds, per token,
+    [kv_compressed | k_pos_emb]; prefill against it uncompresses the cached
+    latents with the kv up-projection (uncompress_kv_from_cache).  [MINIMIND]
+    section 5: with a cache, every history key is visible and the causal mask
+    covers only the new T_q x T_q block.  So, for new token i at position
+    T_past + i:
+
+    1. q and [c | k_pe] of the new tokens as in ``prefill`` (RoPE at
+       positions T_past + i).
+    2. Keys/values of all T_past + T_new positions from the latent rows
+       [past_cache | RMSNorm(c_new) | roped k_pe_new] uncompressed by kv_b.
+    3. softmax over keys 0 .. T_past + i, then o_proj.
+
+    ``past_cache``: [B, T_past, kv_lora_rank + rope] (already normalised and
+    roped).  ``inp``: PrefillInputs of the new tokens (inp.T = T_new).
+    """
+    B, Tn = inp.B, inp.T
+    H, h = cfg.hidden_size, cfg.num_heads
+    dn, dr, dv = cfg.qk_nope_head_dim, cfg.qk_rope_head_dim, cfg.v_head_dim
+    dq = dn + dr
+    r_kv = cfg.kv_lora_rank
+    eps = cfg.rms_eps
+    scale = softmax_scale(cfg)
+    Ta = T_past + Tn
+    x = _f64(inp.x).reshape(B, Tn, H)
+    past = _f64(past_cache).reshape(B, T_past, r_kv + dr)
+
+    kva = x @ _f64(inp.w_kv_a).T
+    c, kpe = kva[..., :r_kv], kva[..., r_kv:]
+    c_hat = rms_norm(c, _f64(inp.g_kv_a), eps)
+    if cfg.q_lora_rank > 0:
+        q = rms_norm(x @ _f64(inp.w_q_a).T, _f64(inp.g_q_a), eps) @ _f64(inp.w_q_b).T
+    else:
+        q = x @ _f64(inp.w_q).T
+    q = q.reshape(B, Tn, h, dq)
+    q_nope, q_pe = q[..., :dn], q[..., dn:]
+    if cfg.rope_type != "none":
+        cos, sin = rope_tables(cfg, Ta)
+        cn, sn = cos[T_past:Ta], sin[T_past:Ta]
+        kpe = apply_rope(kpe, cn[None], sn[None])
+        q_pe = apply_rope(q_pe, cn[None, :, None, :], sn[None, :, None, :])
+    latent = np.concatenate([past, np.concatenate([c_hat, kpe], -1)], axis=1)
+    kv = (latent[..., :r_kv] @ _f64(inp.w_kv_b).T).reshape(B, Ta, h, dn + dv)
+    k_nope, v = kv[..., :dn], kv[..., dn:]
+    k_pe = latent[..., r_kv:]
+    o = np.empty((B, Tn, h, dv))
+    qpos = T_past + np.arange(Tn)
+    mask = np.arange(Ta)[None, :] > qpos[:, None]
+    for b in range(B):
+        for hh in range(h):
+            Qh = np.concatenate([q_nope[b, :, hh, :], q_pe[b, :, hh, :]], -1)
+            Kh = np.concatenate([k_nope[b, :, hh, :], k_pe[b]], -1)
+            s = np.where(mask, -np.inf, scale * (Qh @ Kh.T))
+            o[b, :, hh, :] = _softmax_rows(s) @ v[b, :, hh, :]
+    out = o.reshape(B, Tn, h * dv) @ _f64(inp.w_o).T
+    if not return_parts:
+        return out
+    return out, dict(attn=o, latent=latent, new_cache=latent[:, T_past:])
+
+
+# ---------------------------------------------------------------------------
 # Decode over the latent cache (D1 .. D4)
 # ---------------------------------------------------------------------------
 def _split_kv_b(cfg, w_kv_b):

@@ -359,3 +359,39 @@ def test_planted_absorption_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(O, "_split_kv_b", orig)
     u = O.decode_unabsorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)
     assert np.max(np.abs(a - u)) > 1e-6
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill against a cached latent (Megatron 推理优化 uncompress;
+# MiniMind section 5: history keys fully visible, new block causal)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("rope", ["plain", "none"])
+@pytest.mark.parametrize("T_past,T_new", [(0, 5), (3, 4), (6, 1)])
+def test_chunked_prefill_equals_full_prefill_rows(rope, T_past, T_new):
+    cfg = tiny_cfg(rope_type=rope)
+    full = make_prefill_inputs(cfg, 2, T_past + T_new, seed=16, gamma="random",
+                               w_std=0.4)
+    out_full, P = O.prefill(cfg, full, return_parts=True)
+    past = P["latent_cache"][:, :T_past]
+    new = type(full)(**{**full.__dict__, "x": full.x[:, T_past:], "T": T_new})
+    out, Q = O.prefill_chunked(cfg, new, past, T_past, return_parts=True)
+    np.testing.assert_allclose(out, out_full[:, T_past:], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(Q["new_cache"], P["latent_cache"][:, T_past:],
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_chunked_prefill_sees_all_history():
+    # with zero queries every visible key has equal weight: the output of
+    # new token i is the mean of V over positions 0 .. T_past + i
+    cfg = tiny_cfg(q_lora_rank=0)
+    T_past, T_new = 4, 3
+    full = make_prefill_inputs(cfg, 1, T_past + T_new, seed=17, w_std=0.4)
+    full.w_q.zero_()
+    _, P = O.prefill(cfg, full, return_parts=True)
+    new = type(full)(**{**full.__dict__, "x": full.x[:, T_past:], "T": T_new})
+    _, Q = O.prefill_chunked(cfg, new, P["latent_cache"][:, :T_past], T_past,
+                             return_parts=True)
+    v = P["v"][0]
+    for i in range(T_new):
+        np.testing.assert_allclose(Q["attn"][0, i], v[:T_past + i + 1].mean(0),
+                                   rtol=1e-12, atol=1e-14)
