@@ -287,6 +287,16 @@ MLA_API mla_status mla_check_device_status(void* workspace, void* stream);
  * mla_kernel_launches -- number of CUDA kernels this library has launched in
  * this process (all threads), for counting launches in a timed region.
  */
+/*
+ * mla_selftest_wait_timeout -- failure-detection self-test (no counterpart in
+ * the pages).  Enqueues one small kernel whose single mbarrier wait can never
+ * be satisfied; the wait gives up after the library's bounded-wait limit
+ * (about 2 s), records MLA_ERR_DEVICE_TIMEOUT in the status word at the start
+ * of `workspace` (>= 256 bytes, 256-byte aligned) and returns, leaving the
+ * context usable.  The status is read with mla_check_device_status.  Nothing
+ * traps, faults or hangs.
+ */
+MLA_API mla_status mla_selftest_wait_timeout(void* workspace, void* stream);
 MLA_API mla_status mla_set_stage_events(void* const* events, int32_t n);
 MLA_API int64_t mla_kernel_launches(void);
 

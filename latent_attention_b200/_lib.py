@@ -26,7 +26,7 @@ EXPORTED = ["mla_abi_version", "mla_status_string", "mla_last_error_detail",
             "mla_prefill_forward", "mla_decode_workspace_size",
             "mla_decode_absorbed", "mla_check_device_status",
             "mla_set_stage_events", "mla_kernel_launches",
-            "mla_decode_absorbed_noalloc"]
+            "mla_decode_absorbed_noalloc", "mla_selftest_wait_timeout"]
 
 
 class mla_config(C.Structure):
@@ -102,6 +102,8 @@ def load():
     lib.mla_set_stage_events.argtypes = [C.POINTER(vp), i32]
     lib.mla_kernel_launches.restype = C.c_int64
     lib.mla_kernel_launches.argtypes = []
+    lib.mla_selftest_wait_timeout.restype = C.c_int
+    lib.mla_selftest_wait_timeout.argtypes = [vp, vp]
     lib.mla_decode_absorbed_noalloc.restype = C.c_int
     lib.mla_decode_absorbed_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, i32, vp,
                                                 vp, vp]

@@ -186,3 +186,21 @@ def test_decode_bad_context_is_flagged(cuda):
     with pytest.raises(MlaError, match="MLA_ERR_SHAPE"):
         dec.check_status()
     dec.check_status()                       # the word was cleared
+
+
+def test_bounded_wait_times_out_and_reports(cuda):
+    """A device wait that nothing satisfies gives up after its bound, sets the
+    status word, and leaves the context usable (failure detection without a
+    GPU fault)."""
+    import time
+    from latent_attention_b200 import MlaError, mla_check_device_status, _lib
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda)
+    lib = _lib.load()
+    t0 = time.time()
+    assert lib.mla_selftest_wait_timeout(ws.data_ptr(), None) == 0
+    with pytest.raises(MlaError, match="MLA_ERR_DEVICE_TIMEOUT"):
+        mla_check_device_status(ws, torch.cuda.default_stream())
+    assert 1.0 < time.time() - t0 < 30.0
+    mla_check_device_status(ws, torch.cuda.default_stream())     # cleared
+    x = torch.ones(4, device=cuda)                               # context still fine
+    assert float((x + 1).sum()) == 8.0
