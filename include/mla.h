@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 1
+#define MLA_ABI_VERSION 2
 
 /* Exported symbols keep default visibility even when the library is built
  * with -fvisibility=hidden. */
@@ -129,9 +129,12 @@ typedef struct mla_weights {
  *   ckv    [N, kv_lora+rope]      gain-scaled latent before the RMS row
  *                                 scale | roped k_pe
  *   attn   [N, heads, v]          attention output before o_proj
+ *   latent [B*(T_past+T), kv_lora+rope]  (mla_prefill_chunked only) the
+ *                                 normalised latent rows of history and new
+ *                                 tokens; kv then covers these rows
  * Offsets are -1 for buffers a configuration does not use. */
 typedef struct mla_prefill_layout {
-  int64_t status, ssq_q, ssq_kv, q_a, ckv, q, kv, attn, total_bytes;
+  int64_t status, ssq_q, ssq_kv, q_a, ckv, q, kv, attn, total_bytes, latent;
 } mla_prefill_layout;
 
 /* Byte offsets of the decode intermediates inside the workspace:
@@ -217,6 +220,42 @@ MLA_API mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights*
                                void* out, void* latent_cache_out,
                                void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/* Workspace bytes mla_prefill_chunked needs; 0 if the arguments are invalid. */
+MLA_API size_t mla_prefill_chunked_workspace_size(const mla_config* cfg, int32_t B,
+                                                  int32_t T_new, int32_t T_past,
+                                                  mla_prefill_layout* layout);
+
+/*
+ * mla_prefill_chunked -- prefill of T_new new tokens per sequence after T_past
+ * tokens that are already in the compressed latent cache.
+ *
+ * [MEGATRON] 推理优化: with cache_mla_latents the cache keeps per token
+ * [kv_compressed | k_pos_emb], and prefill against cached latents
+ * uncompresses them through the kv up-projection (uncompress_kv_from_cache).
+ * [MINIMIND] section 5: with a cache every history key is visible and only
+ * the new T_q x T_q block is causally masked.  So new token i (position
+ * T_past + i) attends to keys 0 .. T_past + i, whose k_nope / V are
+ * kv_b_proj of the latent rows [past_cache | RMSNorm_kv(c_new)] and whose
+ * shared rope key is the cached / newly roped k_pe.  Everything else is
+ * mla_prefill_forward's computation (RoPE of the new tokens at positions
+ * T_past + i).  T_past = 0 is exactly mla_prefill_forward.
+ *
+ *   x            [B, T_new, hidden] (new tokens)
+ *   past_cache   [B, T_past, kv_lora_rank + rope] (NULL when T_past = 0),
+ *                rows as written by latent_cache_out of an earlier call
+ *   rope_cos/sin fp32 [>= T_past + T_new, rope]
+ *   out          [B, T_new, hidden]
+ *   latent_cache_out  NULL or [B*T_new, kv_lora_rank + rope]: the new tokens'
+ *                cache rows (append them to the history for the next chunk)
+ *   workspace    >= mla_prefill_chunked_workspace_size bytes, 256-aligned
+ */
+MLA_API mla_status mla_prefill_chunked(const mla_config* cfg, const mla_weights* w,
+                                       const void* x, int32_t B, int32_t T_new,
+                                       const void* past_cache, int32_t T_past,
+                                       const float* rope_cos, const float* rope_sin,
+                                       void* out, void* latent_cache_out, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /* Workspace bytes mla_decode_absorbed needs for (cfg, B, max_ctx); 0 if the
  * arguments are invalid.  Fills *layout when it is not NULL. */

@@ -16,6 +16,7 @@ __all__ = ["MlaError", "make_config", "mla_build_rope_tables",
            "mla_prefill_workspace_size", "mla_prefill_forward",
            "mla_decode_workspace_size", "mla_decode_absorbed",
            "mla_check_device_status", "mla_decode_absorbed_noalloc",
+           "mla_prefill_chunked_workspace_size", "mla_prefill_chunked",
            "abi_version"]
 
 
@@ -106,6 +107,40 @@ def mla_prefill_forward(cfg, weights, x, B, T, rope_cos, rope_sin, out,
         _ptr(workspace, "workspace"), C.c_size_t(workspace.numel() *
                                                  workspace.element_size()),
         _stream(stream)))
+
+
+def mla_prefill_chunked_workspace_size(cfg, B, T_new, T_past):
+    c = cfg if isinstance(cfg, mla_config) else make_config(cfg)
+    lay = mla_prefill_layout()
+    n = _lib.load().mla_prefill_chunked_workspace_size(
+        C.byref(c), int(B), int(T_new), int(T_past), C.byref(lay))
+    if n == 0:
+        raise MlaError(2, "invalid configuration or sizes")
+    return n, {f: getattr(lay, f) for f, _ in lay._fields_}
+
+
+def _weights(weights):
+    w = mla_weights()
+    for f, _ in w._fields_:
+        t = weights.get(f) if hasattr(weights, "get") else getattr(weights, f)
+        setattr(w, f, None if t is None else _ptr(t, f).value)
+    return w
+
+
+def mla_prefill_chunked(cfg, weights, x, B, T_new, past_cache, T_past, rope_cos,
+                        rope_sin, out, workspace, latent_cache_out=None,
+                        stream=None):
+    """Prefill of T_new tokens after T_past tokens held in ``past_cache``
+    ([B, T_past, kv_lora_rank + rope], the latent cache rows)."""
+    c = cfg if isinstance(cfg, mla_config) else make_config(cfg)
+    w = _weights(weights)
+    _check(_lib.load().mla_prefill_chunked(
+        C.byref(c), C.byref(w), _ptr(x, "x"), int(B), int(T_new),
+        _ptr(past_cache, "past_cache", True), int(T_past),
+        _ptr(rope_cos, "rope_cos", True), _ptr(rope_sin, "rope_sin", True),
+        _ptr(out, "out"), _ptr(latent_cache_out, "latent_cache_out", True),
+        _ptr(workspace, "workspace"),
+        C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
 
 
 def mla_decode_workspace_size(cfg, B, max_ctx):

@@ -95,9 +95,13 @@ struct PrefillPlan {
   int N;
 };
 
-void prefill_layout(const mla_config& c, int B, int T, mla_prefill_layout* L) {
-  const int64_t N = (int64_t)B * T, es = elem_size(c);
+// Prefill workspace for B sequences of T new tokens after T_past cached ones
+// (T_past = 0: plain prefill).  Buffers over the new tokens are N = B*T rows;
+// with a cache, the full latent rows and kv cover B*(T_past + T) rows.
+void prefill_layout(const mla_config& c, int B, int T, int T_past, mla_prefill_layout* L) {
+  const int64_t N = (int64_t)B * T, Na = (int64_t)B * (T + T_past), es = elem_size(c);
   const int dq = c.qk_nope_head_dim + c.qk_rope_head_dim;
+  const int w = c.kv_lora_rank + c.qk_rope_head_dim;
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off = align256(off + bytes); return o; };
   L->status = take(256);
@@ -106,9 +110,10 @@ void prefill_layout(const mla_config& c, int B, int T, mla_prefill_layout* L) {
   L->ssq_q = c.q_lora_rank > 0 ? take(N * 4 * ((c.q_lora_rank + 63) / 64)) : -1;
   L->ssq_kv = take(N * 4 * ((c.kv_lora_rank + 63) / 64));
   L->q_a = c.q_lora_rank > 0 ? take(N * c.q_lora_rank * es) : -1;
-  L->ckv = take(N * (c.kv_lora_rank + c.qk_rope_head_dim) * es);
+  L->ckv = take(N * w * es);
+  L->latent = T_past > 0 ? take(Na * w * es) : -1;
   L->q = take(N * c.num_heads * dq * es);
-  L->kv = take(N * c.num_heads * (c.qk_nope_head_dim + c.v_head_dim) * es);
+  L->kv = take(Na * c.num_heads * (c.qk_nope_head_dim + c.v_head_dim) * es);
   L->attn = take(N * c.num_heads * c.v_head_dim * es);
   L->total_bytes = off;
 }
@@ -135,6 +140,186 @@ void decode_layout(const mla_config& c, int B, int max_ctx, mla_decode_layout* L
 }
 
 char* at(void* ws, int64_t off) { return off < 0 ? nullptr : static_cast<char*>(ws) + off; }
+
+}  // namespace
+
+namespace {
+// Prefill of B sequences of T new tokens after T_past tokens whose latent
+// rows are in past_cache ([B, T_past, r_kv + rope]; T_past = 0: plain).
+mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* x, int32_t B,
+                       int32_t T, const void* past_cache, int32_t T_past,
+                       const float* rope_cos, const float* rope_sin, void* out,
+                       void* latent_cache_out, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  mla_status s = check_config(cfg);
+  if (s != MLA_OK) return s;
+  const mla_config& c = *cfg;
+  if (!w) return fail(MLA_ERR_NULL, "weights is NULL");
+  if (!x || !out || !workspace) return fail(MLA_ERR_NULL, "x/out/workspace is NULL");
+  const bool lora = c.q_lora_rank > 0;
+  if (lora && (!w->w_q_a || !w->w_q_b)) return fail(MLA_ERR_NULL, "w_q_a/w_q_b is NULL (q_lora_rank > 0)");
+  if (!lora && !w->w_q) return fail(MLA_ERR_NULL, "w_q is NULL (q_lora_rank == 0)");
+  if (!w->w_kv_a || !w->w_kv_b || !w->w_o) return fail(MLA_ERR_NULL, "w_kv_a/w_kv_b/w_o is NULL");
+  const bool rope = c.rope_type != MLA_ROPE_NONE;
+  if (rope && (!rope_cos || !rope_sin)) return fail(MLA_ERR_NULL, "rope_cos/rope_sin is NULL");
+  if (B < 1 || T < 1 || T_past < 0 || (int64_t)B * ((int64_t)T + T_past) >= (1ll << 31))
+    return fail(MLA_ERR_SHAPE, "B=%d T=%d T_past=%d", B, T, T_past);
+  const void* ptrs[] = {x, out, latent_cache_out, w->w_q_a, w->g_q_a, w->w_q_b, w->w_q,
+                        w->w_kv_a, w->g_kv_a, w->w_kv_b, w->w_o, rope_cos, rope_sin, past_cache};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(MLA_ERR_ALIGN, "pointer %p is not 16-byte aligned", p);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(MLA_ERR_ALIGN, "workspace is not 256-byte aligned");
+  mla_prefill_layout L;
+  prefill_layout(c, B, T, T_past, &L);
+  if ((int64_t)workspace_bytes < L.total_bytes)
+    return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
+                (long long)L.total_bytes);
+
+  const int N = B * T;
+  const int Ta = T + T_past;                    // keys per sequence
+  const int h = c.num_heads, dn = c.qk_nope_head_dim, dr = c.qk_rope_head_dim, dv = c.v_head_dim;
+  const int dq = dn + dr, r_kv = c.kv_lora_rank, H = c.hidden_size;
+  const float eps = (float)c.rms_eps;
+  const bool tc_attn = mla::tc_attention_supported(c);
+  if (rope && (!rope_fits_simt_tiles(dq, dn, dr, h) ||
+               !rope_fits_simt_tiles(r_kv + dr, r_kv, dr, 1)) && c.dtype == MLA_F32)
+    return fail(MLA_ERR_UNSUPPORTED, "rope columns straddle a 64-column tile");
+  if (!tc_attn &&
+      sizeof(float) * (16 * dq + 32 * dq + 32 * dv + 16 * 32 + 16 * dv + 48) > 227 * 1024)
+    return fail(MLA_ERR_UNSUPPORTED, "head dims too large for the CUDA-core attention");
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = static_cast<char*>(workspace);
+  float* ssq_q = (float*)at(ws, L.ssq_q);
+  float* ssq_kv = (float*)at(ws, L.ssq_kv);
+  void* q_a = at(ws, L.q_a);
+  void* ckv = at(ws, L.ckv);
+  void* q = at(ws, L.q);
+  void* kv = at(ws, L.kv);
+  void* attn = at(ws, L.attn);
+  void* latent = at(ws, L.latent);
+  uint32_t* status = (uint32_t*)at(ws, L.status);
+
+  // The status word starts at zero; every other buffer is fully written.
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  mla::stage_event(0, st);
+
+  // S1: fused down-projection [x W_qa^T | x W_kva^T]; epilogue: RMS row
+  // statistics, gains, RoPE on k_pe.
+  mla::GemmArgs g;
+  g.A = x; g.lda = H; g.M = N; g.K = H;
+  int si = 0;
+  if (lora) {
+    mla::EpiSeg& e0 = g.seg[si];
+    g.Bm[si] = w->w_q_a; g.ldb[si] = H;
+    e0.out = q_a; e0.ldo = c.q_lora_rank; e0.ncols = c.q_lora_rank;
+    e0.gamma = w->g_q_a; e0.norm_cols = c.q_lora_rank; e0.ssq_out = ssq_q; e0.ssq_ld = N;
+    ++si;
+  }
+  {
+    mla::EpiSeg& e1 = g.seg[si];
+    g.Bm[si] = w->w_kv_a; g.ldb[si] = H;
+    e1.out = ckv; e1.ldo = r_kv + dr; e1.ncols = r_kv + dr;
+    e1.gamma = w->g_kv_a; e1.norm_cols = r_kv; e1.ssq_out = ssq_kv; e1.ssq_ld = N;
+    if (rope) {
+      e1.cos = rope_cos; e1.sin = rope_sin; e1.rope_period = r_kv + dr;
+      e1.rope_start = r_kv; e1.rope_dim = dr; e1.T = T; e1.pos_offset = T_past;
+    }
+    ++si;
+  }
+  g.nseg = si;
+  // Each projection runs on the tensor-core GEMM when it takes the shape;
+  // the column tile of the down-projection fixes the RMS partial count.
+  auto run_gemm = [&](const mla::GemmArgs& ga) {
+    if (mla::tc_gemm_supported(ga, c.dtype)) return mla::tc_gemm(ga, st, status);
+    if (ga.seg[0].cos && !rope_fits_simt_tiles(ga.seg[0].rope_period, ga.seg[0].rope_start,
+                                               ga.seg[0].rope_dim,
+                                               ga.seg[0].ncols / ga.seg[0].rope_period))
+      return cudaErrorNotSupported;
+    return mla::launch_gemm_simt(c.dtype, ga, st);
+  };
+  const int tile_n = mla::tc_gemm_supported(g, c.dtype) ? mla::kTcTileN : mla::kSimtTileN;
+  e = run_gemm(g);
+  if (e != cudaSuccess) return cuda_fail(e, "down-projection");
+  mla::stage_event(1, st);
+
+  // S2+S3: q up-projection (RMS row scale) or direct q_proj; RoPE on q_pe.
+  mla::GemmArgs gq;
+  gq.M = N; gq.nseg = 1;
+  mla::EpiSeg& eq = gq.seg[0];
+  if (lora) {
+    gq.A = q_a; gq.lda = c.q_lora_rank; gq.K = c.q_lora_rank;
+    gq.Bm[0] = w->w_q_b; gq.ldb[0] = c.q_lora_rank;
+    eq.ssq_in = ssq_q; eq.rs_inv_dim = 1.0f / c.q_lora_rank; eq.eps = eps;
+    eq.ssq_parts = (c.q_lora_rank + tile_n - 1) / tile_n; eq.ssq_ld = N;
+  } else {
+    gq.A = x; gq.lda = H; gq.K = H;
+    gq.Bm[0] = w->w_q; gq.ldb[0] = H;
+  }
+  eq.out = q; eq.ldo = (int64_t)h * dq; eq.ncols = h * dq;
+  if (rope) {
+    eq.cos = rope_cos; eq.sin = rope_sin; eq.rope_period = dq; eq.rope_start = dn;
+    eq.rope_dim = dr; eq.T = T; eq.pos_offset = T_past;
+  }
+  e = run_gemm(gq);
+  if (e != cudaSuccess) return cuda_fail(e, "q projection");
+  mla::stage_event(2, st);
+
+  // S2+S4: kv up-projection.  Plain prefill: straight from the gain-scaled
+  // latent with the kv RMS row scale in the epilogue.  With a cache: over the
+  // full latent rows [past | RMSNorm(c_new) | k_pe] (the uncompress step),
+  // which are normalised already.
+  const void* kv_src = ckv;
+  if (T_past > 0) {
+    const size_t row = (size_t)(r_kv + dr) * elem_size(c);
+    e = cudaMemcpy2DAsync(latent, (size_t)Ta * row, past_cache, (size_t)T_past * row,
+                          (size_t)T_past * row, (size_t)B, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "latent history copy");
+    e = mla::launch_latent_finalize(c.dtype, ckv, ssq_kv, (r_kv + tile_n - 1) / tile_n, N, r_kv,
+                                    dr, eps, latent, st, T, Ta, T_past);
+    if (e != cudaSuccess) return cuda_fail(e, "latent assembly");
+    kv_src = latent;
+  }
+  mla::GemmArgs gk;
+  gk.A = kv_src; gk.lda = r_kv + dr; gk.M = B * Ta; gk.K = r_kv; gk.nseg = 1;
+  gk.Bm[0] = w->w_kv_b; gk.ldb[0] = r_kv;
+  mla::EpiSeg& ek = gk.seg[0];
+  ek.out = kv; ek.ldo = (int64_t)h * (dn + dv); ek.ncols = h * (dn + dv);
+  if (T_past == 0) {
+    ek.ssq_in = ssq_kv; ek.rs_inv_dim = 1.0f / r_kv; ek.eps = eps;
+    ek.ssq_parts = (r_kv + tile_n - 1) / tile_n; ek.ssq_ld = N;
+  }
+  e = run_gemm(gk);
+  if (e != cudaSuccess) return cuda_fail(e, "kv up-projection");
+  mla::stage_event(3, st);
+
+  // S7: causal attention (new queries at positions T_past .. T_past + T - 1).
+  mla::AttnArgs aa{q, kv, kv_src, attn, B, T, h, dn, dr, dv, r_kv, (float)softmax_scale(c), status};
+  aa.Tk = Ta;
+  aa.q_off = T_past;
+  e = tc_attn ? mla::tc_attention(aa, st) : mla::launch_attn_simt(c.dtype, aa, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  mla::stage_event(4, st);
+
+  // S8: o_proj.
+  mla::GemmArgs go;
+  go.A = attn; go.lda = (int64_t)h * dv; go.M = N; go.K = h * dv; go.nseg = 1;
+  go.Bm[0] = w->w_o; go.ldb[0] = (int64_t)h * dv;
+  go.seg[0].out = out; go.seg[0].ldo = H; go.seg[0].ncols = H;
+  e = run_gemm(go);
+  if (e != cudaSuccess) return cuda_fail(e, "o_proj");
+  mla::stage_event(5, st);
+
+  if (latent_cache_out) {
+    e = mla::launch_latent_finalize(c.dtype, ckv, ssq_kv, (r_kv + tile_n - 1) / tile_n, N, r_kv,
+                                    dr, eps, latent_cache_out, st);
+    if (e != cudaSuccess) return cuda_fail(e, "latent cache");
+  }
+  g_detail.clear();
+  return MLA_OK;
+}
+
 
 }  // namespace
 
@@ -195,7 +380,7 @@ size_t mla_prefill_workspace_size(const mla_config* cfg, int32_t B, int32_t T,
                                   mla_prefill_layout* layout) {
   if (check_config(cfg) != MLA_OK || B < 1 || T < 1 || (int64_t)B * T >= (1ll << 31)) return 0;
   mla_prefill_layout L;
-  prefill_layout(*cfg, B, T, &L);
+  prefill_layout(*cfg, B, T, 0, &L);
   if (layout) *layout = L;
   return (size_t)L.total_bytes;
 }
@@ -204,152 +389,30 @@ mla_status mla_prefill_forward(const mla_config* cfg, const mla_weights* w, cons
                                int32_t B, int32_t T, const float* rope_cos,
                                const float* rope_sin, void* out, void* latent_cache_out,
                                void* workspace, size_t workspace_bytes, void* stream) {
-  mla_status s = check_config(cfg);
-  if (s != MLA_OK) return s;
-  const mla_config& c = *cfg;
-  if (!w) return fail(MLA_ERR_NULL, "weights is NULL");
-  if (!x || !out || !workspace) return fail(MLA_ERR_NULL, "x/out/workspace is NULL");
-  const bool lora = c.q_lora_rank > 0;
-  if (lora && (!w->w_q_a || !w->w_q_b)) return fail(MLA_ERR_NULL, "w_q_a/w_q_b is NULL (q_lora_rank > 0)");
-  if (!lora && !w->w_q) return fail(MLA_ERR_NULL, "w_q is NULL (q_lora_rank == 0)");
-  if (!w->w_kv_a || !w->w_kv_b || !w->w_o) return fail(MLA_ERR_NULL, "w_kv_a/w_kv_b/w_o is NULL");
-  const bool rope = c.rope_type != MLA_ROPE_NONE;
-  if (rope && (!rope_cos || !rope_sin)) return fail(MLA_ERR_NULL, "rope_cos/rope_sin is NULL");
-  if (B < 1 || T < 1 || (int64_t)B * T >= (1ll << 31)) return fail(MLA_ERR_SHAPE, "B=%d T=%d", B, T);
-  const void* ptrs[] = {x, out, latent_cache_out, w->w_q_a, w->g_q_a, w->w_q_b, w->w_q,
-                        w->w_kv_a, w->g_kv_a, w->w_kv_b, w->w_o, rope_cos, rope_sin};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return fail(MLA_ERR_ALIGN, "pointer %p is not 16-byte aligned", p);
-  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
-    return fail(MLA_ERR_ALIGN, "workspace is not 256-byte aligned");
+  return run_prefill(cfg, w, x, B, T, nullptr, 0, rope_cos, rope_sin, out, latent_cache_out,
+                     workspace, workspace_bytes, stream);
+}
+
+size_t mla_prefill_chunked_workspace_size(const mla_config* cfg, int32_t B, int32_t T_new,
+                                          int32_t T_past, mla_prefill_layout* layout) {
+  if (check_config(cfg) != MLA_OK || B < 1 || T_new < 1 || T_past < 0 ||
+      (int64_t)B * ((int64_t)T_new + T_past) >= (1ll << 31))
+    return 0;
   mla_prefill_layout L;
-  prefill_layout(c, B, T, &L);
-  if ((int64_t)workspace_bytes < L.total_bytes)
-    return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
-                (long long)L.total_bytes);
+  prefill_layout(*cfg, B, T_new, T_past, &L);
+  if (layout) *layout = L;
+  return (size_t)L.total_bytes;
+}
 
-  const int N = B * T;
-  const int h = c.num_heads, dn = c.qk_nope_head_dim, dr = c.qk_rope_head_dim, dv = c.v_head_dim;
-  const int dq = dn + dr, r_kv = c.kv_lora_rank, H = c.hidden_size;
-  const float eps = (float)c.rms_eps;
-  const bool tc_attn = mla::tc_attention_supported(c);
-  if (rope && (!rope_fits_simt_tiles(dq, dn, dr, h) ||
-               !rope_fits_simt_tiles(r_kv + dr, r_kv, dr, 1)) && c.dtype == MLA_F32)
-    return fail(MLA_ERR_UNSUPPORTED, "rope columns straddle a 64-column tile");
-  if (!tc_attn &&
-      sizeof(float) * (16 * dq + 32 * dq + 32 * dv + 16 * 32 + 16 * dv + 48) > 227 * 1024)
-    return fail(MLA_ERR_UNSUPPORTED, "head dims too large for the CUDA-core attention");
-  cudaStream_t st = (cudaStream_t)stream;
-  char* ws = static_cast<char*>(workspace);
-  float* ssq_q = (float*)at(ws, L.ssq_q);
-  float* ssq_kv = (float*)at(ws, L.ssq_kv);
-  void* q_a = at(ws, L.q_a);
-  void* ckv = at(ws, L.ckv);
-  void* q = at(ws, L.q);
-  void* kv = at(ws, L.kv);
-  void* attn = at(ws, L.attn);
-  uint32_t* status = (uint32_t*)at(ws, L.status);
-
-  // The status word starts at zero; every other buffer is fully written.
-  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
-  if (e != cudaSuccess) return cuda_fail(e, "memset");
-  mla::stage_event(0, st);
-
-  // S1: fused down-projection [x W_qa^T | x W_kva^T]; epilogue: RMS row
-  // statistics, gains, RoPE on k_pe.
-  mla::GemmArgs g;
-  g.A = x; g.lda = H; g.M = N; g.K = H;
-  int si = 0;
-  if (lora) {
-    mla::EpiSeg& e0 = g.seg[si];
-    g.Bm[si] = w->w_q_a; g.ldb[si] = H;
-    e0.out = q_a; e0.ldo = c.q_lora_rank; e0.ncols = c.q_lora_rank;
-    e0.gamma = w->g_q_a; e0.norm_cols = c.q_lora_rank; e0.ssq_out = ssq_q; e0.ssq_ld = N;
-    ++si;
-  }
-  {
-    mla::EpiSeg& e1 = g.seg[si];
-    g.Bm[si] = w->w_kv_a; g.ldb[si] = H;
-    e1.out = ckv; e1.ldo = r_kv + dr; e1.ncols = r_kv + dr;
-    e1.gamma = w->g_kv_a; e1.norm_cols = r_kv; e1.ssq_out = ssq_kv; e1.ssq_ld = N;
-    if (rope) {
-      e1.cos = rope_cos; e1.sin = rope_sin; e1.rope_period = r_kv + dr;
-      e1.rope_start = r_kv; e1.rope_dim = dr; e1.T = T;
-    }
-    ++si;
-  }
-  g.nseg = si;
-  // Each projection runs on the tensor-core GEMM when it takes the shape;
-  // the column tile of the down-projection fixes the RMS partial count.
-  auto run_gemm = [&](const mla::GemmArgs& ga) {
-    if (mla::tc_gemm_supported(ga, c.dtype)) return mla::tc_gemm(ga, st, status);
-    if (ga.seg[0].cos && !rope_fits_simt_tiles(ga.seg[0].rope_period, ga.seg[0].rope_start,
-                                               ga.seg[0].rope_dim,
-                                               ga.seg[0].ncols / ga.seg[0].rope_period))
-      return cudaErrorNotSupported;
-    return mla::launch_gemm_simt(c.dtype, ga, st);
-  };
-  const int tile_n = mla::tc_gemm_supported(g, c.dtype) ? mla::kTcTileN : mla::kSimtTileN;
-  e = run_gemm(g);
-  if (e != cudaSuccess) return cuda_fail(e, "down-projection");
-  mla::stage_event(1, st);
-
-  // S2+S3: q up-projection (RMS row scale) or direct q_proj; RoPE on q_pe.
-  mla::GemmArgs gq;
-  gq.M = N; gq.nseg = 1;
-  mla::EpiSeg& eq = gq.seg[0];
-  if (lora) {
-    gq.A = q_a; gq.lda = c.q_lora_rank; gq.K = c.q_lora_rank;
-    gq.Bm[0] = w->w_q_b; gq.ldb[0] = c.q_lora_rank;
-    eq.ssq_in = ssq_q; eq.rs_inv_dim = 1.0f / c.q_lora_rank; eq.eps = eps;
-    eq.ssq_parts = (c.q_lora_rank + tile_n - 1) / tile_n; eq.ssq_ld = N;
-  } else {
-    gq.A = x; gq.lda = H; gq.K = H;
-    gq.Bm[0] = w->w_q; gq.ldb[0] = H;
-  }
-  eq.out = q; eq.ldo = (int64_t)h * dq; eq.ncols = h * dq;
-  if (rope) {
-    eq.cos = rope_cos; eq.sin = rope_sin; eq.rope_period = dq; eq.rope_start = dn;
-    eq.rope_dim = dr; eq.T = T;
-  }
-  e = run_gemm(gq);
-  if (e != cudaSuccess) return cuda_fail(e, "q projection");
-  mla::stage_event(2, st);
-
-  // S2+S4: kv up-projection with the kv RMS row scale.
-  mla::GemmArgs gk;
-  gk.A = ckv; gk.lda = r_kv + dr; gk.M = N; gk.K = r_kv; gk.nseg = 1;
-  gk.Bm[0] = w->w_kv_b; gk.ldb[0] = r_kv;
-  mla::EpiSeg& ek = gk.seg[0];
-  ek.out = kv; ek.ldo = (int64_t)h * (dn + dv); ek.ncols = h * (dn + dv);
-  ek.ssq_in = ssq_kv; ek.rs_inv_dim = 1.0f / r_kv; ek.eps = eps;
-  ek.ssq_parts = (r_kv + tile_n - 1) / tile_n; ek.ssq_ld = N;
-  e = run_gemm(gk);
-  if (e != cudaSuccess) return cuda_fail(e, "kv up-projection");
-  mla::stage_event(3, st);
-
-  // S7: causal attention.
-  mla::AttnArgs aa{q, kv, ckv, attn, B, T, h, dn, dr, dv, r_kv, (float)softmax_scale(c), status};
-  e = tc_attn ? mla::tc_attention(aa, st) : mla::launch_attn_simt(c.dtype, aa, st);
-  if (e != cudaSuccess) return cuda_fail(e, "attention");
-  mla::stage_event(4, st);
-
-  // S8: o_proj.
-  mla::GemmArgs go;
-  go.A = attn; go.lda = (int64_t)h * dv; go.M = N; go.K = h * dv; go.nseg = 1;
-  go.Bm[0] = w->w_o; go.ldb[0] = (int64_t)h * dv;
-  go.seg[0].out = out; go.seg[0].ldo = H; go.seg[0].ncols = H;
-  e = run_gemm(go);
-  if (e != cudaSuccess) return cuda_fail(e, "o_proj");
-  mla::stage_event(5, st);
-
-  if (latent_cache_out) {
-    e = mla::launch_latent_finalize(c.dtype, ckv, ssq_kv, (r_kv + tile_n - 1) / tile_n, N, r_kv,
-                                    dr, eps, latent_cache_out, st);
-    if (e != cudaSuccess) return cuda_fail(e, "latent cache");
-  }
-  g_detail.clear();
-  return MLA_OK;
+mla_status mla_prefill_chunked(const mla_config* cfg, const mla_weights* w, const void* x,
+                               int32_t B, int32_t T_new, const void* past_cache,
+                               int32_t T_past, const float* rope_cos, const float* rope_sin,
+                               void* out, void* latent_cache_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (T_past < 0) return fail(MLA_ERR_SHAPE, "T_past=%d", T_past);
+  if (T_past > 0 && !past_cache) return fail(MLA_ERR_NULL, "past_cache is NULL (T_past > 0)");
+  return run_prefill(cfg, w, x, B, T_new, past_cache, T_past, rope_cos, rope_sin, out,
+                     latent_cache_out, workspace, workspace_bytes, stream);
 }
 
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t B, int32_t max_ctx,

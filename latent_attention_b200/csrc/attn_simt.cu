@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnArgs a) {
   const int64_t qstride = (int64_t)a.h * dq;
   const int64_t kvstride = (int64_t)a.h * (a.dn + a.dv);
   const int64_t cstride = a.r_kv + a.dr;
-  const int64_t base = (int64_t)b * a.T;
+  const int64_t base = (int64_t)b * a.T;        // first query row of the sequence
+  const int64_t kbase = (int64_t)b * a.Tk;      // first key row of the sequence
 
   for (int idx = tid; idx < BQ * dq; idx += NT) {
     const int i = idx / dq, d = idx % dq;
@@ -50,30 +51,31 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnArgs a) {
   __syncthreads();
 
   const int q_last = min(q0 + BQ, a.T) - 1;
-  for (int k0 = 0; k0 <= q_last; k0 += BKEY) {
+  const int k_last = min(a.q_off + q_last, a.Tk - 1);
+  for (int k0 = 0; k0 <= k_last; k0 += BKEY) {
     for (int idx = tid; idx < BKEY * dq; idx += NT) {
       const int j = idx / dq, d = idx % dq;
       const int t = k0 + j;
       float v = 0.f;
-      if (t < a.T) {
-        v = d < a.dn ? Elem<T>::load(kv + (base + t) * kvstride + (int64_t)hh * (a.dn + a.dv) + d)
-                     : Elem<T>::load(ckv + (base + t) * cstride + a.r_kv + (d - a.dn));
+      if (t < a.Tk) {
+        v = d < a.dn ? Elem<T>::load(kv + (kbase + t) * kvstride + (int64_t)hh * (a.dn + a.dv) + d)
+                     : Elem<T>::load(ckv + (kbase + t) * cstride + a.r_kv + (d - a.dn));
       }
       Ks[idx] = v;
     }
     for (int idx = tid; idx < BKEY * a.dv; idx += NT) {
       const int j = idx / a.dv, d = idx % a.dv;
       const int t = k0 + j;
-      Vs[idx] = t < a.T ? Elem<T>::load(kv + (base + t) * kvstride +
-                                        (int64_t)hh * (a.dn + a.dv) + a.dn + d)
-                        : 0.f;
+      Vs[idx] = t < a.Tk ? Elem<T>::load(kv + (kbase + t) * kvstride +
+                                         (int64_t)hh * (a.dn + a.dv) + a.dn + d)
+                         : 0.f;
     }
     __syncthreads();
     for (int idx = tid; idx < BQ * BKEY; idx += NT) {
       const int i = idx / BKEY, j = idx % BKEY;
       float s = 0.f;
       for (int d = 0; d < dq; ++d) s = fmaf(Qs[i * dq + d], Ks[j * dq + d], s);
-      const bool masked = (k0 + j > q0 + i) || (k0 + j >= a.T);
+      const bool masked = (k0 + j > a.q_off + q0 + i) || (k0 + j >= a.Tk);
       Ss[idx] = masked ? -INFINITY : s * a.scale;
     }
     __syncthreads();
@@ -113,7 +115,9 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnArgs a) {
 
 }  // namespace
 
-cudaError_t launch_attn_simt(int dtype, const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_attn_simt(int dtype, const AttnArgs& a_in, cudaStream_t st) {
+  AttnArgs a = a_in;
+  if (a.Tk <= 0) a.Tk = a.T;
   const int dq = a.dn + a.dr;
   const size_t smem = sizeof(float) *
       (BQ * dq + BKEY * dq + BKEY * a.dv + BQ * BKEY + BQ * a.dv + 3 * BQ);

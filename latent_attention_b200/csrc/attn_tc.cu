@@ -54,7 +54,8 @@ constexpr uint32_t TM_S = 0, TM_O = 256;                   // + 128 * tile
 constexpr float kRescaleLog2 = 8.f;
 
 struct AttnTcParams {
-  int B, T, h;
+  int B, T, h;           // T queries per sequence
+  int Tk, q_off;         // keys per sequence, position of query 0
   float scale_log2;      // softmax scale * log2(e)
   int n_pairs;           // CTAs per head: ceil(T / 256)
   __nv_bfloat16* o;      // [N, h, DV]
@@ -79,11 +80,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int hh = blockIdx.y % p.h;
   const int b = blockIdx.y / p.h;
   const int c = p.n_pairs - 1 - blockIdx.x;          // heaviest pair first
-  const int row0 = b * p.T;                          // first token of the sequence
-  // tile X covers queries [q0X, q0X + 128) and key blocks [0, nkvX)
+  const int row0 = b * p.T;                          // first query row of the sequence
+  const int krow0 = b * p.Tk;                        // first key row of the sequence
+  // tile X covers queries [q0X, q0X + 128) (positions + q_off) and key
+  // blocks [0, nkvX)
   const int q0A = 256 * c, q0B = 256 * c + BQ;
-  const int nkvA = q0A < p.T ? min(q0A + BQ - 1, p.T - 1) / BKV + 1 : 0;
-  const int nkvB = q0B < p.T ? min(q0B + BQ - 1, p.T - 1) / BKV + 1 : 0;
+  const int nkvA = q0A < p.T ? min(p.q_off + q0A + BQ - 1, p.Tk - 1) / BKV + 1 : 0;
+  const int nkvB = q0B < p.T ? min(p.q_off + q0B + BQ - 1, p.Tk - 1) / BKV + 1 : 0;
   const int nkv = max(nkvA, nkvB);
 
   if (threadIdx.x == 0) {
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&k_empty, (j & 1) ^ 1, abort_v, p.status)) break;
         uint8_t* sk = smem + OFF_K;
         mbar_arrive_expect_tx(&k_full, K_BYTES);
-        const int kr = row0 + j * BKV;
+        const int kr = krow0 + j * BKV;
         tma_load_2d(sk, &tmKV, hh * (DN + DV), kr, &k_full);
         tma_load_2d(sk + BOX, &tmKV, hh * (DN + DV) + 64, kr, &k_full);
         tma_load_2d(sk + 2 * BOX, &tmKpe, 0, kr, &k_full);
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&v_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
         uint8_t* sv = smem + OFF_V + slot * V_BYTES;
         mbar_arrive_expect_tx(&v_full[slot], V_BYTES);
-        const int kr = row0 + j * BKV;
+        const int kr = krow0 + j * BKV;
         tma_load_2d(sv, &tmKV, hh * (DN + DV) + DN, kr, &v_full[slot]);
         tma_load_2d(sv + BOX, &tmKV, hh * (DN + DV) + DN + 64, kr, &v_full[slot]);
       }
@@ -226,7 +229,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, sr[cc]);
       tmem_wait_ld();
       // Raw scores; the scale is folded into the exp argument below (scale > 0).
-      const int kmax = min(qi, p.T - 1) - j * BKV;   // last visible key in this block
+      const int kmax = min(p.q_off + qi, p.Tk - 1) - j * BKV;  // last visible key here
       if (kmax < 127) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
@@ -326,7 +329,9 @@ bool tc_attention_supported(const mla_config& c) {
 }
 
 cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
-  const int64_t N = (int64_t)a.B * a.T;
+  const int64_t N = (int64_t)a.B * a.T;          // query rows
+  const int Tk = a.Tk > 0 ? a.Tk : a.T;
+  const int64_t Nk = (int64_t)a.B * Tk;          // key rows
   CUtensorMap tmQ, tmKV, tmKpe;
   const uint32_t box[2] = {64, 128};
   {
@@ -335,13 +340,13 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
     if (!encode_tmap(&tmQ, a.q, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[2] = {(uint64_t)a.h * (DN + DV), (uint64_t)N};
+    const uint64_t dims[2] = {(uint64_t)a.h * (DN + DV), (uint64_t)Nk};
     const uint64_t strides[1] = {(uint64_t)a.h * (DN + DV) * 2};
     if (!encode_tmap(&tmKV, a.kv, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     // k_pe columns [r_kv, r_kv + 64) of the latent buffer [N, r_kv + 64]
-    const uint64_t dims[2] = {(uint64_t)DR, (uint64_t)N};
+    const uint64_t dims[2] = {(uint64_t)DR, (uint64_t)Nk};
     const uint64_t strides[1] = {(uint64_t)(a.r_kv + a.dr) * 2};
     const __nv_bfloat16* kpe = reinterpret_cast<const __nv_bfloat16*>(a.ckv) + a.r_kv;
     if (!encode_tmap(&tmKpe, kpe, 2, dims, strides, box)) return cudaErrorInvalidValue;
@@ -350,6 +355,8 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
   p.B = a.B;
   p.T = a.T;
   p.h = a.h;
+  p.Tk = Tk;
+  p.q_off = a.q_off;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.n_pairs = (a.T + 2 * BQ - 1) / (2 * BQ);
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);

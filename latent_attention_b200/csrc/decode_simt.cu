@@ -20,19 +20,20 @@ template <typename T>
 __global__ void latent_finalize_kernel(const T* __restrict__ ckv,
                                        const float* __restrict__ ssq, int parts, int N,
                                        int r, int dr, float eps,
-                                       T* __restrict__ cache) {
+                                       T* __restrict__ cache, int Tsrc, int dst_T, int dst_off) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int w = r + dr;
   if (idx >= (int64_t)N * w) return;
   const int64_t m = idx / w;
   const int c = (int)(idx % w);
+  const int64_t drow = (m / Tsrc) * dst_T + dst_off + (m % Tsrc);
   float v = Elem<T>::load(ckv + idx);
   if (c < r) {
     float ss = 0.f;
     for (int p = 0; p < parts; ++p) ss += ssq[(int64_t)p * N + m];
     v *= rsqrtf(ss * (1.0f / r) + eps);
   }
-  Elem<T>::store(cache + idx, v);
+  Elem<T>::store(cache + drow * w + c, v);
 }
 
 // D1: one block per (b, h); q_lat row = [W_UK^T q_nope | q_pe] in fp32 math.
@@ -187,16 +188,18 @@ cudaError_t run_decode(const DecodeArgs& a, cudaStream_t st) {
 
 cudaError_t launch_latent_finalize(int dtype, const void* ckv, const float* ssq_kv,
                                    int ssq_parts, int N, int r_kv, int dr, float eps, void* cache,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, int T, int dst_T, int dst_off) {
   const int64_t total = (int64_t)N * (r_kv + dr);
   const unsigned blocks = (unsigned)((total + 255) / 256);
   count_launches();
   if (dtype == MLA_F32)
     latent_finalize_kernel<float><<<blocks, 256, 0, st>>>(
-        (const float*)ckv, ssq_kv, ssq_parts, N, r_kv, dr, eps, (float*)cache);
+        (const float*)ckv, ssq_kv, ssq_parts, N, r_kv, dr, eps, (float*)cache, T, dst_T,
+        dst_off);
   else
     latent_finalize_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)ckv, ssq_kv, ssq_parts, N, r_kv, dr, eps, (__nv_bfloat16*)cache);
+        (const __nv_bfloat16*)ckv, ssq_kv, ssq_parts, N, r_kv, dr, eps, (__nv_bfloat16*)cache,
+        T, dst_T, dst_off);
   return cudaGetLastError();
 }
 

@@ -36,7 +36,7 @@ template <> struct Elem<__nv_bfloat16> {
 //   v *= rsqrt(sum_p ssq_in[p * ssq_ld + m] * rs_inv_dim + eps)   if ssq_in
 //                                   (RMS row scale; partials summed in order)
 //   RoPE on cols with (n % rope_period) in [rope_start, rope_start+rope_dim)
-//        position = m % T, pairs (i, i + rope_dim/2)            if cos
+//        position = m % T + pos_offset, pairs (i, i + rope_dim/2)  if cos
 //   v *= gamma[n]                   for n < norm_cols           if gamma
 //   out[m * ldo + n] = v (rounded to the element type)
 struct EpiSeg {
@@ -54,6 +54,7 @@ struct EpiSeg {
   const float* cos = nullptr;
   const float* sin = nullptr;
   int rope_period = 0, rope_start = 0, rope_dim = 0, T = 1;
+  int pos_offset = 0;       // RoPE position = (row % T) + pos_offset
 };
 
 // C = A B^T with A [M, K] (row stride lda) and the output columns split in up
@@ -78,14 +79,20 @@ struct GemmArgs {
   bool b_mn = false;
 };
 
+// Causal attention of B sequences: T queries per sequence at positions
+// q_off .. q_off + T - 1 against Tk keys per sequence at positions 0 .. Tk - 1
+// (key j visible to query i iff j <= q_off + i).  Plain prefill: Tk = T,
+// q_off = 0; prefill against a cache of T_past tokens: Tk = T_past + T,
+// q_off = T_past.
 struct AttnArgs {
-  const void* q;        // [N, h, dq]
-  const void* kv;       // [N, h, dn+dv]
-  const void* ckv;      // [N, r_kv+dr]  (k_pe at column r_kv)
-  void* o;              // [N, h, dv]
+  const void* q;        // [B*T, h, dq]
+  const void* kv;       // [B*Tk, h, dn+dv]
+  const void* ckv;      // [B*Tk, r_kv+dr]  (k_pe at column r_kv)
+  void* o;              // [B*T, h, dv]
   int B, T, h, dn, dr, dv, r_kv;
   float scale;
   uint32_t* status;
+  int Tk = 0, q_off = 0;
 };
 
 struct DecodeArgs {
@@ -119,10 +126,13 @@ cudaError_t launch_gemm_simt(int dtype, const GemmArgs& a, cudaStream_t st);
 // Column tile width of the CUDA-core GEMM (RMS partial count = ceil(cols/64)).
 constexpr int kSimtTileN = 64;
 cudaError_t launch_attn_simt(int dtype, const AttnArgs& a, cudaStream_t st);
+// Normalised latent rows [RMSNorm(c) | k_pe] from the gain-scaled latent
+// buffer: source row m (of N = B*T) goes to destination row
+// (m / T) * dst_T + dst_off + (m % T).
 cudaError_t launch_latent_finalize(int dtype, const void* ckv,
                                    const float* ssq_kv, int ssq_parts, int N, int r_kv,
                                    int dr, float eps, void* cache,
-                                   cudaStream_t st);
+                                   cudaStream_t st, int T = 1, int dst_T = 1, int dst_off = 0);
 cudaError_t launch_decode_simt(int dtype, const DecodeArgs& a, cudaStream_t st);
 
 }  // namespace mla

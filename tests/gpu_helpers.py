@@ -54,3 +54,30 @@ def run_decode(cfg, di, max_ctx, with_o=False):
     torch.cuda.synchronize()
     dec.check_status()
     return dec, out
+
+
+def run_prefill_chunked(cfg, inp, past, T_past):
+    """mla_prefill_chunked on the new tokens of ``inp`` after ``past``
+    ([B, T_past, r + rope] on the host, or None)."""
+    from latent_attention_b200 import (make_config, mla_build_rope_tables,
+                                       mla_prefill_chunked,
+                                       mla_prefill_chunked_workspace_size)
+    B, T = inp.B, inp.T
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    c = make_config(cfg)
+    d = cfg.qk_rope_head_dim
+    cos = torch.empty(T_past + T, d, device="cuda")
+    sin = torch.empty_like(cos)
+    mla_build_rope_tables(c, T_past + T, cos, sin)
+    n, lay = mla_prefill_chunked_workspace_size(c, B, T, T_past)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty(B, T, cfg.hidden_size, dtype=dt, device="cuda")
+    cache = torch.empty(B * T, cfg.kv_lora_rank + d, dtype=dt, device="cuda")
+    w = {k: (None if v is None else v.cuda()) for k, v in weights_of(inp).items()}
+    mla_prefill_chunked(c, w, inp.x.cuda(), B, T,
+                        None if past is None else past.cuda().contiguous(), T_past,
+                        cos, sin, out, ws, latent_cache_out=cache)
+    torch.cuda.synchronize()
+    from latent_attention_b200 import mla_check_device_status
+    mla_check_device_status(ws)
+    return out, cache, ws, lay

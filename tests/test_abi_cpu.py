@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 1
+    assert lib.mla_abi_version() == 2
     for code, name in {0: b"MLA_OK", 5: b"MLA_ERR_WORKSPACE",
                        8: b"MLA_ERR_DEVICE_TIMEOUT"}.items():
         assert lib.mla_status_string(code) == name
@@ -65,7 +65,7 @@ int main(void) {
   printf("mla_decode_layout %zu\n", sizeof(mla_decode_layout));
   P(mla_config, rope_theta) P(mla_config, original_max_position_embeddings)
   P(mla_config, dtype) P(mla_config, rms_eps) P(mla_config, softmax_scale)
-  P(mla_weights, w_o) P(mla_decode_layout, split_tokens)
+  P(mla_weights, w_o) P(mla_decode_layout, split_tokens) P(mla_prefill_layout, latent)
   P(mla_decode_layout, max_splits)
   return 0;
 }
@@ -166,3 +166,31 @@ def test_binding_refuses_cpu_tensors(lib):
     t = torch.empty(4, 16)
     with pytest.raises(ValueError, match="CUDA"):
         mla_build_rope_tables(cfg, 4, t, t)
+
+
+def test_chunked_prefill_validation_and_sizes(lib):
+    from latent_attention_b200 import (make_config, mla_weights,
+                                       mla_prefill_workspace_size,
+                                       mla_prefill_chunked_workspace_size)
+    cfg = WORKLOADS["dsv3_prefill"].cfg
+    # no history: the same workspace as a plain prefill
+    n0, _ = mla_prefill_workspace_size(cfg, 2, 300)
+    n1, l1 = mla_prefill_chunked_workspace_size(cfg, 2, 300, 0)
+    assert n0 == n1 and l1["latent"] == -1
+    # history: latent rows and kv cover T_past + T_new rows per sequence
+    n2, l2 = mla_prefill_chunked_workspace_size(cfg, 2, 300, 1000)
+    w = cfg.kv_lora_rank + cfg.qk_rope_head_dim
+    assert l2["latent"] >= 0 and n2 >= n1 + 2 * 1300 * w * 2
+    c = make_config(cfg)
+    wt = mla_weights()
+    for i, f in enumerate(("w_q_a", "g_q_a", "w_q_b", "w_kv_a", "g_kv_a",
+                           "w_kv_b", "w_o")):
+        setattr(wt, f, 0x100000 + i * 0x1000)
+    p, ws, big = _fake(0x200000), _fake(0x1000000), C.c_size_t(1 << 40)
+    f = lib.mla_prefill_chunked
+    assert f(C.byref(c), C.byref(wt), p, 1, 8, None, 4, p, p, p, None, ws, big,
+             None) == 1                                 # history without cache
+    assert f(C.byref(c), C.byref(wt), p, 1, 8, p, -1, p, p, p, None, ws, big,
+             None) == 2
+    assert f(C.byref(c), C.byref(wt), p, 1, 8, _fake(0x200008), 4, p, p, p, None,
+             ws, big, None) == 3

@@ -204,3 +204,65 @@ def test_bounded_wait_times_out_and_reports(cuda):
     mla_check_device_status(ws, torch.cuda.default_stream())     # cleared
     x = torch.ones(4, device=cuda)                               # context still fine
     assert float((x + 1).sum()) == 8.0
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill against a cached latent
+# --------------------------------------------------------------------------
+CHUNKED = [
+    ("tiny_f32", W["tiny_f32"].cfg, 2, 40, 25),
+    ("tiny_f32_nopast", W["tiny_f32"].cfg, 1, 30, 0),
+    ("bf16_dsv3dims", small_bf16(), 2, 130, 257),
+    ("bf16_one_token", small_bf16(), 3, 1, 300),
+    ("bf16_kimi_norope", small_bf16(rope_type="none", num_heads=3), 1, 200, 64),
+    ("bf16_directq", small_bf16(q_lora_rank=0, rope_type="plain", num_heads=2),
+     2, 64, 129),
+]
+
+
+@pytest.mark.parametrize("name,cfg,B,T_new,T_past", CHUNKED,
+                         ids=[c[0] for c in CHUNKED])
+def test_prefill_chunked_small(cuda, name, cfg, B, T_new, T_past):
+    from gpu_helpers import run_prefill_chunked
+    inp = make_prefill_inputs(cfg, B, T_new, seed=21, gamma="random")
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    g = torch.Generator().manual_seed(22)
+    past = (torch.randn(B, T_past, cfg.kv_lora_rank + cfg.qk_rope_head_dim,
+                        generator=g).to(dt) if T_past else None)
+    out, cache, _, _ = run_prefill_chunked(cfg, inp, past, T_past)
+    ref, P = oracle.prefill_chunked(
+        cfg, inp, past if past is not None else
+        torch.zeros(B, 0, cfg.kv_lora_rank + cfg.qk_rope_head_dim), T_past,
+        return_parts=True)
+    tol = TOL[cfg.dtype]
+    assert oracle.max_rel_err(out, ref) <= tol
+    assert oracle.max_rel_err(cache.view(B, T_new, -1), P["new_cache"]) <= tol
+
+
+def test_prefill_chunked_composes_with_prefill(cuda):
+    """prefill of the first T_past tokens (its latent cache output) followed by
+    a chunked prefill of the rest matches one prefill over all tokens."""
+    from gpu_helpers import run_prefill_chunked
+    cfg = small_bf16()
+    B, T_past, T_new = 2, 200, 120
+    full = make_prefill_inputs(cfg, B, T_past + T_new, seed=23)
+    first = type(full)(**{**full.__dict__, "x": full.x[:, :T_past], "T": T_past})
+    rest = type(full)(**{**full.__dict__, "x": full.x[:, T_past:], "T": T_new})
+    _, _, cache = run_prefill(cfg, first)
+    out_c, _, _, _ = run_prefill_chunked(cfg, rest, cache.view(B, T_past, -1).cpu(),
+                                         T_past)
+    _, out_f, _ = run_prefill(cfg, full, latent=False)
+    assert oracle.max_rel_err(out_c, out_f[:, T_past:]) <= TOL["bf16"]
+
+
+def test_prefill_chunked_dsv3_heads(cuda):
+    from gpu_helpers import run_prefill_chunked
+    cfg = W["dsv3_prefill"].cfg
+    B, T_new, T_past = 1, 256, 1024
+    inp = make_prefill_inputs(cfg, B, T_new, seed=24)
+    g = torch.Generator().manual_seed(25)
+    past = torch.randn(B, T_past, cfg.kv_lora_rank + cfg.qk_rope_head_dim,
+                       generator=g).to(torch.bfloat16)
+    out, _, _, _ = run_prefill_chunked(cfg, inp, past, T_past)
+    ref = oracle.prefill_chunked(cfg, inp, past, T_past)
+    assert oracle.max_rel_err(out, ref) <= TOL["bf16"]
