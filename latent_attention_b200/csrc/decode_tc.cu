@@ -18,17 +18,20 @@
 // scores.  A cluster of two CTAs therefore shares one (sequence, split):
 // CTA c holds latent columns [256c, 256c+256) of O (256 TMEM columns) and
 // contracts the scores over its share of the 576 cached dims -- CTA 0 over
-// dims [0, 256), CTA 1 over [256, 576) (latent half + the 64 rope dims).
-// Each CTA TMA-loads only its own dims of every 64-token chunk, so every
-// cache byte crosses HBM once; the same shared-memory tile is the K-major B
-// operand of S = Q C^T and the MN-major B operand of O += P C.  The two
-// partial score tiles (fp32, 128 x 64) are exchanged through distributed
-// shared memory; both CTAs add them in the same order and run the identical
-// online softmax, so P, the running max and the row sums agree bit for bit
-// without further exchange.  Warp roles (256 threads per CTA):
-//   warp 0     TMA: Q share once, chunk ring (2 stages), L2 prefetch ahead
-//   warp 1     TMEM allocation, MMA issue (S_j, then O += P_{j-1} C_{j-1})
-//   warps 2, 3, 8, 9  score exchange, one chunk ahead of the softmax
+// dims [0, 256), CTA 1 over [256, 576) (latent half + the 64 rope dims, whose
+// query part sits in TMEM).  Each CTA TMA-loads only its own dims of every
+// 64-token chunk, so every cache byte crosses HBM once; the same shared-memory
+// tile is the K-major B operand of S = Q C^T and the MN-major B operand of
+// O += P C.  The partial score tiles are exchanged through distributed shared
+// memory as fp16; each CTA adds the peer's partial to its own fp32 one and runs
+// the online softmax for all 128 heads.  The MMA warp issues the scores two
+// chunks ahead of the PV product (three chunk stages, three score slots), so
+// the exchange and softmax of chunk j overlap the tensor work of j+1 and j+2.
+// P_j (bf16 pairs) is written over the first half of S_j's TMEM slot.
+// Warp roles (320 threads per CTA):
+//   warp 0     TMA: Q share once, chunk ring (3 stages), L2 prefetch ahead
+//   warp 1     TMEM allocation, MMA issue (S_j, then O += P_{j-2} C_{j-2})
+//   warps 2, 3, 8, 9  score exchange (fp16 partial to the peer)
 //   warps 4-7  softmax (thread = head), P into TMEM, epilogue
 // All waits are bounded; a timeout sets the device status word.
 #include <cfloat>
@@ -46,24 +49,27 @@ constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row widt
 constexpr int NT = 64;                           // tokens per chunk
 constexpr int QBOX = 128 * 64 * 2;               // 128 heads x 64 dims bf16
 constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
-constexpr int MAX_ATOMS = 5;
+constexpr int QATOMS = 4;                        // latent dims of Q in shared memory
+constexpr int MAX_ATOMS = 5;                     // cache atoms per chunk (CTA 1: + rope)
+constexpr int NSTAGE = 3;                        // chunk ring / score slots
 constexpr int OFF_Q = 0;
-constexpr int OFF_C = OFF_Q + MAX_ATOMS * QBOX;          // 80 KB
+constexpr int OFF_C = OFF_Q + QATOMS * QBOX;             // 64 KB
 constexpr int STAGE = MAX_ATOMS * CBOX;                  // 40 KB
 constexpr int XBUF = 128 * NT * 2;                       // exchange: 128 x 64 fp16
-constexpr int OFF_X = OFF_C + 2 * STAGE;                 // two exchange buffers
+constexpr int OFF_X = OFF_C + NSTAGE * STAGE;            // peer partials received (x2)
 constexpr int SMEM_BYTES = OFF_X + 2 * XBUF + 1024;
 constexpr int NTHREADS = 320;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
-// TMEM: S slots [0, 128), P slots (128 rows x 64 keys bf16 = 32 columns each)
-// [128, 192), O [256, 512).
-constexpr uint32_t TM_S = 0, TM_P = 128, TM_O = 256;
+// TMEM: score slots [0, 192) (64 columns each; P_j over the first 32 of slot
+// j % 3), rope part of Q on CTA 1 [192, 224), O [256, 512).
+constexpr uint32_t TM_S = 0, TM_QPE = 192, TM_O = 256;
 constexpr float kRescaleLog2 = 8.f;
 
 struct DecTcParams {
   const int32_t* cu_ctx;
+  const __nv_bfloat16* q_pe;   // [B, h, 64]
   int B, h, max_ctx;
   int split_tokens, max_splits;
   float scale_log2;
@@ -105,14 +111,26 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
   return __half22float2(*reinterpret_cast<__half2*>(&v));
 }
 
+// S_j = Q_share C_j^T over the ATOMS 64-dim atoms held in shared memory.
+// Descriptors advance by their 16-byte address field only (shared-memory
+// addresses stay below 2^18, so the field never carries).
+template <int ATOMS>
+__device__ __forceinline__ void issue_scores(uint32_t d_tmem, uint64_t dq, uint64_t dc) {
+#pragma unroll
+  for (int a = 0; a < ATOMS; ++a)
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      mma_bf16(d_tmem, dq + (uint64_t)((a * QBOX + k * 32) >> 4),
+               dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, (a | k) != 0);
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
-                       const __grid_constant__ CUtensorMap tmQpe,
                        const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, c_full[2], c_empty[2], s_full[2], s_comb[2],
-      s_free[2], p_full, pv_done[2], x_full[2], x_empty[2];
+  __shared__ __align__(8) uint64_t q_full, qpe_full, c_full[NSTAGE], c_empty[NSTAGE],
+      s_full[NSTAGE], s_free[NSTAGE], p_full[NSTAGE], pv_done[2], o_done, x_full[2], x_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -135,24 +153,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
   const int tcount = min(p.split_tokens, n - t0);
   const int nch = (tcount + NT - 1) / NT;
-  const int atoms = rank == 0 ? 4 : 5;
+  const bool rope = rank == 1;
+  const int atoms = rope ? 5 : 4;
   const int dim0 = 256 * (int)rank;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    mbar_init(&qpe_full, 4);        // softmax warps stored the rope query (CTA 1)
+    for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&c_full[s], 1);
       mbar_init(&c_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_comb[s], 4);
-      mbar_init(&s_free[s], 4);
+      mbar_init(&s_free[s], 4);     // exchange warps have read S_j from TMEM
+      mbar_init(&p_full[s], 4);     // softmax warps have written P_j
     }
-    mbar_init(&p_full, 4);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
+    mbar_init(&o_done, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&x_full[s], 1);    // one local arrive.expect_tx + the peer's st.async bytes
-      mbar_init(&x_empty[s], 4);   // one arrive per exchange warp of the peer
+      mbar_init(&x_empty[s], 4);   // one arrive per softmax warp of the peer
     }
     abort_flag = 0;
     fence_barrier_init();
@@ -172,174 +192,187 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     if (elect_one()) {
       tma_prefetch(&tmQ);
-      tma_prefetch(&tmQpe);
       tma_prefetch(&tmC);
-      mbar_arrive_expect_tx(&q_full, atoms * QBOX);
-      for (int a = 0; a < 4; ++a)
+      mbar_arrive_expect_tx(&q_full, QATOMS * QBOX);
+      for (int a = 0; a < QATOMS; ++a)
         tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, dim0 + 64 * a, b * p.h + h0, &q_full);
-      if (atoms == 5)
-        tma_load_2d(smem + OFF_Q + 4 * QBOX, &tmQpe, 0, b * p.h + h0, &q_full);
       for (int j = 0; j < PREFETCH && j < nch; ++j)
         for (int a = 0; a < atoms; ++a)
           tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, (int)start + chunk_base(n, t0, j));
       for (int j = 0; j < nch; ++j) {
-        const int slot = j & 1;
+        const int st = j % NSTAGE;
         if (j + PREFETCH < nch)
           for (int a = 0; a < atoms; ++a)
             tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, (int)start + chunk_base(n, t0, j + PREFETCH));
-        if (!mbar_wait(&c_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
-        uint8_t* sc = smem + OFF_C + slot * STAGE;
-        mbar_arrive_expect_tx(&c_full[slot], atoms * CBOX);
+        if (!mbar_wait(&c_empty[st], ((j / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+        uint8_t* sc = smem + OFF_C + st * STAGE;
+        mbar_arrive_expect_tx(&c_full[st], atoms * CBOX);
         const int y = (int)start + chunk_base(n, t0, j);
         for (int a = 0; a < atoms; ++a)
-          tma_load_2d(sc + a * CBOX, &tmC, dim0 + 64 * a, y, &c_full[slot]);
+          tma_load_2d(sc + a * CBOX, &tmC, dim0 + 64 * a, y, &c_full[st]);
       }
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t sq = smem_u32(smem + OFF_Q);
+      const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_Q));
       bool ok = mbar_wait(&q_full, 0, abort_v, p.status);
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&p_full, j & 1, abort_v, p.status)) return false;
-        tc_fence_after();
-        const uint32_t sc = smem_u32(smem + OFF_C + (j & 1) * STAGE);
+      if (ok && rope) ok = mbar_wait(&qpe_full, 0, abort_v, p.status);
+      for (int j = 0; ok && j < nch + 2; ++j) {
+        if (j < nch) {   // S_j into slot j % 3
+          const int st = j % NSTAGE;
+          if (!mbar_wait(&c_full[st], (j / NSTAGE) & 1, abort_v, p.status)) break;
+          // the slot's previous scores S_{j-3} were read by the exchange warps;
+          // its P_{j-3} was consumed by PV_{j-3}, issued before this point
+          if (j >= NSTAGE &&
+              !mbar_wait(&s_free[st], ((j - NSTAGE) / NSTAGE) & 1, abort_v, p.status))
+            break;
+          tc_fence_after();
+          const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
+          issue_scores<QATOMS>(tbase + TM_S + st * NT, dq, dc);
+          if (rope) {
 #pragma unroll
-        for (int k = 0; k < NT / 16; ++k)   // A = P_j from TMEM slot j % 2, 8 columns per step
-          mma_bf16_ts(tbase + TM_O, tbase + TM_P + (j & 1) * 32 + k * 8,
-                      desc_mnmajor_sw128(sc + k * 16 * 128, CBOX), IDESC_PV, (j | k) != 0);
-        mma_commit(&c_empty[j & 1]);
-        mma_commit(&pv_done[j & 1]);
-        return true;
-      };
-      for (int j = 0; ok && j < nch; ++j) {
-        const int slot = j & 1;
-        if (!mbar_wait(&c_full[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
-        if (!mbar_wait(&s_free[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sc = smem_u32(smem + OFF_C + slot * STAGE);
-        for (int a = 0; a < atoms; ++a)
+            for (int k = 0; k < 4; ++k)   // A = rope query from TMEM, 8 columns per K step
+              mma_bf16_ts(tbase + TM_S + st * NT, tbase + TM_QPE + k * 8,
+                          dc + (uint64_t)((QATOMS * CBOX + k * 32) >> 4), IDESC_S, 1);
+          }
+          mma_commit(&s_full[st]);
+        }
+        if (j >= 2) {    // O += P_{j-2} C_{j-2}
+          const int jj = j - 2, st = jj % NSTAGE;
+          if (!mbar_wait(&p_full[st], (jj / NSTAGE) & 1, abort_v, p.status)) break;
+          tc_fence_after();
+          const uint64_t dv = desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE), CBOX);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tbase + TM_S + slot * NT, desc_kmajor_sw128(sq + a * QBOX + k * 32),
-                     desc_kmajor_sw128(sc + a * CBOX + k * 32), IDESC_S, (a | k) != 0);
-        mma_commit(&s_full[slot]);
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+          for (int k = 0; k < NT / 16; ++k)
+            mma_bf16_ts(tbase + TM_O, tbase + TM_S + st * NT + k * 8,
+                        dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (jj | k) != 0);
+          mma_commit(&c_empty[st]);
+          mma_commit(&pv_done[jj & 1]);
+          if (jj == nch - 1) mma_commit(&o_done);
+        }
       }
-      if (ok) issue_pv(nch - 1);
     }
   } else if (xwg) {
-    // ---------------- score exchange: own partial (fp16) to the peer, peer's
-    // partial back, merged scores (fp32) written over the TMEM slot.
+    // ---------------- score exchange: this CTA's partial S_j as fp16 pairs
+    // into the peer's receive buffer j % 2 (rows of this warp's lane quarter).
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     for (int j = 0; j < nch; ++j) {
-      const int slot = j & 1;
-      // exchange buffer j % 2: the peer's send of chunk j only needs this
-      // CTA to have consumed chunk j - 2 from the same buffer
-      const uint32_t sx = smem_u32(smem + OFF_X + slot * XBUF);
-      const uint32_t px = map_peer(sx, peer);
-      const uint32_t px_full = map_peer(smem_u32(&x_full[slot]), peer);
-      const uint32_t px_empty = map_peer(smem_u32(&x_empty[slot]), peer);
-      if (!warp_wait(&s_full[slot], (j >> 1) & 1, abort_v, p.status)) break;
+      const int st = j % NSTAGE, xs = j & 1;
+      const uint32_t px = map_peer(smem_u32(smem + OFF_X + xs * XBUF), peer);
+      const uint32_t px_full = map_peer(smem_u32(&x_full[xs]), peer);
+      if (!warp_wait(&s_full[st], (j / NSTAGE) & 1, abort_v, p.status)) break;
       tc_fence_after();
       uint32_t sr[2][32];
-      tmem_ld32(tbase + lane_off + TM_S + slot * NT, sr[0]);
-      tmem_ld32(tbase + lane_off + TM_S + slot * NT + 32, sr[1]);
+      tmem_ld32(tbase + lane_off + TM_S + st * NT, sr[0]);
+      tmem_ld32(tbase + lane_off + TM_S + st * NT + 32, sr[1]);
       tmem_wait_ld();
-      uint32_t h[32];                                 // own partial as fp16 pairs
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      uint32_t h[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i)
         h[i] = pack_half2(__uint_as_float(sr[i >> 4][(2 * i) & 31]),
                           __uint_as_float(sr[i >> 4][(2 * i + 1) & 31]));
-      if (!warp_wait_cluster(&x_empty[slot], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
+      // the peer's receive buffer j % 2 is free once its softmax consumed j - 2
+      if (!warp_wait_cluster(&x_empty[xs], ((j >> 1) & 1) ^ 1, abort_v, p.status)) break;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         st_async_v4(px + r * 128 + ((c ^ (r & 7)) << 4), h[4 * c], h[4 * c + 1], h[4 * c + 2],
                     h[4 * c + 3], px_full);
-      if (r == 0) mbar_arrive_expect_tx(&x_full[slot], XBUF);
-      if (!warp_wait_cluster(&x_full[slot], (j >> 1) & 1, abort_v, p.status)) break;
-      uint32_t o[2][32];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float a0, a1, a2, a3;
-        ld_shared_v4(sx + r * 128 + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
-        const uint32_t pk[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
-                                __float_as_uint(a3)};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * c + e;                    // half2 index -> scores 2i, 2i+1
-          const float2 mine = unpack_half2(h[i]);
-          const float2 theirs = unpack_half2(pk[e]);
-          // both CTAs add the same two fp16-rounded halves: identical sums
-          o[(2 * i) >> 5][(2 * i) & 31] = __float_as_uint(mine.x + theirs.x);
-          o[(2 * i + 1) >> 5][(2 * i + 1) & 31] = __float_as_uint(mine.y + theirs.y);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote_relaxed(px_empty);
-      tmem_st32(tbase + lane_off + TM_S + slot * NT, o[0]);
-      tmem_st32(tbase + lane_off + TM_S + slot * NT + 32, o[1]);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_comb[slot]);
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- softmax (thread = head) + epilogue
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const int head = h0 + r;
+    const bool head_ok = head < p.h;
+    if (rope) {      // rope part of this head's query into TMEM (A operand layout)
+      uint32_t q[32];
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_pe + ((int64_t)b * p.h + head) * DR);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = head_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        q[4 * c] = v.x;
+        q[4 * c + 1] = v.y;
+        q[4 * c + 2] = v.z;
+        q[4 * c + 3] = v.w;
+      }
+      tmem_st32(tbase + lane_off + TM_QPE, q);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qpe_full);
+    }
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
-      const int slot = j & 1;
-      if (!warp_wait(&s_comb[slot], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
+      const int st = j % NSTAGE, xs = j & 1;
+      if (!warp_wait(&s_full[st], (j / NSTAGE) & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[2][32];
-      tmem_ld32(tbase + lane_off + TM_S + slot * NT, sr[0]);
-      tmem_ld32(tbase + lane_off + TM_S + slot * NT + 32, sr[1]);
+      tmem_ld32(tbase + lane_off + TM_S + st * NT, sr[0]);
+      tmem_ld32(tbase + lane_off + TM_S + st * NT + 32, sr[1]);
+      if (r == 0) mbar_arrive_expect_tx(&x_full[xs], XBUF);
+      if (!warp_wait_cluster(&x_full[xs], (j >> 1) & 1, abort_v, p.status)) { ok = false; break; }
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[slot]);
+      // S_j = own fp32 partial + the peer's fp16 partial
+      const uint32_t sx = smem_u32(smem + OFF_X + xs * XBUF);
+      float s[NT];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t t[4];
+        ld_shared_v4u(sx + r * 128 + ((c ^ (r & 7)) << 4), t[0], t[1], t[2], t[3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 8 * c + 2 * e;
+          const float2 theirs = unpack_half2(t[e]);
+          float s0 = __uint_as_float(sr[i >> 5][i & 31]);
+          float s1 = __uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]);
+          add2(s0, s1, theirs.x, theirs.y);
+          s[i] = s0;
+          s[i + 1] = s1;
+        }
+      }
       // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
       const int lo = j * NT - (chunk_base(n, t0, j) - t0);
       const int hi = tcount - (chunk_base(n, t0, j) - t0);
-      float s[NT];
-      float mx8[8];
+      // Raw scores; the (positive) scale is folded into the exp argument.
+      if (lo > 0 || hi < NT) {       // first / last chunk of the split only
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        const float v = __uint_as_float(sr[i >> 5][i & 31]) * p.scale_log2;
-        s[i] = (i >= lo && i < hi) ? v : -INFINITY;
-        mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+        for (int i = 0; i < NT; ++i)
+          if (i < lo || i >= hi) s[i] = -INFINITY;
       }
-      const float mx = fmaxf(m_ref, fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))));
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < NT; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], s[i], s[i + 1]);
+      const float mx = fmaxf(m_ref, max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * p.scale_log2);
       const bool grow = mx > m_ref + kRescaleLog2;
       const float alpha = grow ? ex2(m_ref - mx) : 1.f;
       if (grow) {
         l *= alpha;
         m_ref = mx;
       }
+      const float neg_m = -m_ref;
       float ls[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
       uint32_t w[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2(s[2 * e] - m_ref);
-        const float p1 = ex2(s[2 * e + 1] - m_ref);
-        ls[e & 7] += p0 + p1;
+        float a0, a1;
+        fma2(a0, a1, s[2 * e], s[2 * e + 1], p.scale_log2, p.scale_log2, neg_m, neg_m);
+        const float p0 = ex2(a0);
+        const float p1 = ex2(a1);
+        add2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
         w[e] = pack_bf16(p0, p1);
       }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      // A rescale of O needs every earlier PV finished (PV_{j-1} is the last);
-      // otherwise only the PV that read this P slot two chunks ago must be done.
-      const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
-      if (rescale) {
+      // A rescale of O needs every earlier PV finished; PV_{j-1} is the last.
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
         if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
           ok = false;
           break;
@@ -354,23 +387,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tbase + lane_off + TM_O + c * 32, o);
         }
-      } else if (j > 1) {
-        if (!warp_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
       }
-      tmem_st32(tbase + lane_off + TM_P + (j & 1) * 32, w);
+      // P_j goes over S_j: this CTA's exchange warps must have read S_j.
+      if (!warp_wait(&s_free[st], (j / NSTAGE) & 1, abort_v, p.status)) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32(tbase + lane_off + TM_S + st * NT, w);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full);
+      if (lane == 0) {
+        mbar_arrive(&p_full[st]);
+        // The receive buffer of chunk j is consumed: every value loaded from
+        // it fed P_j, whose TMEM store has completed.
+        mbar_arrive_remote_relaxed(map_peer(smem_u32(&x_empty[xs]), peer));
+      }
     }
-    if (ok && warp_wait(&pv_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_v, p.status)) {
+    if (ok && warp_wait(&o_done, 0, abort_v, p.status)) {
       tc_fence_after();
-      const int head = h0 + r;
-      const bool head_ok = head < p.h;
       const int64_t part = ((int64_t)b * p.max_splits + sp) * p.h + head;
       const float inv = 1.f / l;
       float* dst = p.part_o + part * R + dim0;
@@ -457,14 +490,11 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
   stage_event(1, st);
   // D2
   {
-    CUtensorMap tmQ, tmQpe, tmC;
+    CUtensorMap tmQ, tmC;
     const uint32_t qbox[2] = {64, 128}, cbox[2] = {64, NT};
     const uint64_t qdims[2] = {(uint64_t)R, (uint64_t)a.B * a.h};
     const uint64_t qstr[1] = {(uint64_t)R * 2};
     if (!encode_tmap(&tmQ, a.q_lat, 2, qdims, qstr, qbox)) return cudaErrorInvalidValue;
-    const uint64_t pdims[2] = {(uint64_t)DR, (uint64_t)a.B * a.h};
-    const uint64_t pstr[1] = {(uint64_t)DR * 2};
-    if (!encode_tmap(&tmQpe, a.q_pe, 2, pdims, pstr, qbox)) return cudaErrorInvalidValue;
     // The cache holds sum(ctx) <= B * max_ctx rows; cu_ctx lives on the
     // device, so the map is declared with the bound and every box is clamped
     // inside its own sequence (chunk_base).
@@ -473,6 +503,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
     if (!encode_tmap(&tmC, a.cache, 2, cdims, cstr, cbox)) return cudaErrorInvalidValue;
     DecTcParams p{};
     p.cu_ctx = a.cu_ctx;
+    p.q_pe = reinterpret_cast<const __nv_bfloat16*>(a.q_pe);
     p.B = a.B;
     p.h = a.h;
     p.max_ctx = a.max_ctx;
@@ -490,7 +521,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
       attr = true;
     }
     dim3 grid(2 * a.B * a.max_splits, 1, (a.h + 127) / 128);
-    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, p);
+    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmC, p);
     count_launches();
   }
   stage_event(2, st);
