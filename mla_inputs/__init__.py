@@ -6,8 +6,9 @@ draw the very same inputs from it without sharing any computation.
 """
 from .configs import MlaConfig, WORKLOADS, workload
 from .generate import (PrefillInputs, DecodeInputs, make_prefill_inputs,
-                       make_decode_inputs, decode_context_lengths)
+                       make_decode_inputs, decode_context_lengths,
+                       varlen_seq_lengths, make_varlen_inputs)
 
 __all__ = ["MlaConfig", "WORKLOADS", "workload", "PrefillInputs",
            "DecodeInputs", "make_prefill_inputs", "make_decode_inputs",
-           "decode_context_lengths"]
+           "decode_context_lengths", "varlen_seq_lengths", "make_varlen_inputs"]

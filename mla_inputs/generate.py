@@ -82,6 +82,25 @@ def make_prefill_inputs(cfg: MlaConfig, B: int, T: int, seed: int = 0,
                          w_o, B, T)
 
 
+def varlen_seq_lengths(n_seq: int, len_min: int, len_max: int,
+                       seed: int = 0) -> torch.Tensor:
+    """Lengths of packed prefill sequences, uniform on [len_min, len_max]."""
+    g = _gen(seed + 6007)
+    return torch.randint(len_min, len_max + 1, (n_seq,), generator=g,
+                         dtype=torch.int64).to(torch.int32)
+
+
+def make_varlen_inputs(cfg: MlaConfig, seq_lengths, seed: int = 0,
+                       gamma: str = "ones"):
+    """Packed (THD) prefill inputs: the sequences' tokens back to back as one
+    PrefillInputs with B = 1, T = sum(lengths), plus int32 cu_seqlens [n+1]."""
+    lens = torch.as_tensor(seq_lengths, dtype=torch.int64).reshape(-1)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lens, 0)
+    inp = make_prefill_inputs(cfg, 1, int(cu[-1]), seed=seed, gamma=gamma)
+    return inp, cu.to(torch.int32)
+
+
 def decode_context_lengths(B: int, ctx_min: int, ctx_max: int,
                            seed: int = 0) -> torch.Tensor:
     """Per-sequence cached context lengths, uniform on [ctx_min, ctx_max]."""

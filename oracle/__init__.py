@@ -22,13 +22,17 @@ Functions and what pins them (tests/test_oracle_pins.py):
   with the last row of a prefill.
 * ``prefill_chunked`` -- equals the last rows of a full prefill whose first
   positions produced the cache; reduces to ``prefill`` with no history.
+* ``prefill_varlen`` -- equals separate ``prefill`` calls on each packed
+  sequence (block-diagonal mask vs separate problems); one sequence reduces
+  to ``prefill``; one-token sequences return their own value row.
 """
 from .mla_oracle import (yarn_get_mscale, softmax_scale, rope_frequencies,
                          rope_tables, rms_norm, rotate_half, apply_rope,
-                         prefill, prefill_chunked, decode_absorbed,
+                         prefill, prefill_chunked, prefill_varlen,
+                         decode_absorbed,
                          decode_unabsorbed, max_rel_err)
 
 __all__ = ["yarn_get_mscale", "softmax_scale", "rope_frequencies",
            "rope_tables", "rms_norm", "rotate_half", "apply_rope", "prefill",
-           "prefill_chunked",
+           "prefill_chunked", "prefill_varlen",
            "decode_absorbed", "decode_unabsorbed", "max_rel_err"]

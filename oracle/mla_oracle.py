@@ -330,6 +330,67 @@ def prefill_chunked(cfg, inp, past_cache, T_past: int,
     return out, dict(attn=o, latent=latent, new_cache=latent[:, T_past:])
 
 
+def _packed_rows(cu_seqlens, N):
+    """Sequence index b(m) and in-sequence position of every packed row."""
+    cu = np.asarray(_f64(cu_seqlens), dtype=np.int64)
+    assert cu[0] == 0 and cu[-1] == N and np.all(np.diff(cu) >= 0)
+    seq = np.searchsorted(cu, np.arange(N), side="right") - 1
+    return seq, np.arange(N) - cu[seq]
+
+
+def prefill_varlen(cfg, inp, cu_seqlens, return_parts: bool = False):
+    """Packed (THD) prefill: ``inp.x`` holds N tokens of several sequences back
+    to back, sequence b owning rows cu_seqlens[b] .. cu_seqlens[b+1]-1.
+
+    [MEGATRON] 训练支持与并行策略 packs variable-length sequences in the THD
+    layout described by cumulative sequence lengths.  Every step of
+    ``prefill`` is per token except RoPE and attention, so in packed form:
+    the position of row m is m - cu_seqlens[b(m)] (positions restart at 0 in
+    every sequence), and query m attends to key k only when both rows belong
+    to the same sequence and pos(k) <= pos(m) (a block-diagonal causal mask
+    over the packed rows).
+
+    ``inp``: PrefillInputs with B = 1, T = N.  Returns out [N, hidden] and, on
+    request, the parts (attention output, latent cache rows).
+    """
+    N = inp.T
+    H, h = cfg.hidden_size, cfg.num_heads
+    dn, dr, dv = cfg.qk_nope_head_dim, cfg.qk_rope_head_dim, cfg.v_head_dim
+    dq = dn + dr
+    r_kv = cfg.kv_lora_rank
+    eps = cfg.rms_eps
+    scale = softmax_scale(cfg)
+    seq, pos = _packed_rows(cu_seqlens, N)
+
+    x = _f64(inp.x).reshape(N, H)
+    kva = x @ _f64(inp.w_kv_a).T
+    c, kpe = kva[:, :r_kv], kva[:, r_kv:]
+    c_hat = rms_norm(c, _f64(inp.g_kv_a), eps)
+    kv = (c_hat @ _f64(inp.w_kv_b).T).reshape(N, h, dn + dv)
+    k_nope, v = kv[..., :dn], kv[..., dn:]
+    if cfg.q_lora_rank > 0:
+        q = rms_norm(x @ _f64(inp.w_q_a).T, _f64(inp.g_q_a), eps) @ _f64(inp.w_q_b).T
+    else:
+        q = x @ _f64(inp.w_q).T
+    q = q.reshape(N, h, dq)
+    q_nope, q_pe = q[..., :dn], q[..., dn:]
+    if cfg.rope_type != "none":
+        cos, sin = rope_tables(cfg, int(pos.max()) + 1 if N else 1)
+        kpe = apply_rope(kpe, cos[pos], sin[pos])
+        q_pe = apply_rope(q_pe, cos[pos][:, None, :], sin[pos][:, None, :])
+    visible = (seq[None, :] == seq[:, None]) & (pos[None, :] <= pos[:, None])
+    o = np.empty((N, h, dv))
+    for hh in range(h):
+        Qh = np.concatenate([q_nope[:, hh, :], q_pe[:, hh, :]], -1)
+        Kh = np.concatenate([k_nope[:, hh, :], kpe], -1)
+        s = np.where(visible, scale * (Qh @ Kh.T), -np.inf)
+        o[:, hh, :] = _softmax_rows(s) @ v[:, hh, :]
+    out = o.reshape(N, h * dv) @ _f64(inp.w_o).T
+    if not return_parts:
+        return out
+    return out, dict(attn=o, latent_cache=np.concatenate([c_hat, kpe], -1), pos=pos, seq=seq)
+
+
 # ---------------------------------------------------------------------------
 # Decode over the latent cache (D1 .. D4)
 # ---------------------------------------------------------------------------

@@ -395,3 +395,67 @@ def test_chunked_prefill_sees_all_history():
     for i in range(T_new):
         np.testing.assert_allclose(Q["attn"][0, i], v[:T_past + i + 1].mean(0),
                                    rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Packed (THD) prefill (Megatron 训练支持与并行策略: cu_seqlens packing)
+# --------------------------------------------------------------------------
+def _sequence_inputs(inp, lo, hi):
+    """PrefillInputs of packed rows lo..hi-1 as one B=1 sequence."""
+    return type(inp)(**{**inp.__dict__, "x": inp.x[:, lo:hi], "T": hi - lo})
+
+
+@pytest.mark.parametrize("rope,q_lora", [("plain", 8), ("none", 0)])
+def test_varlen_prefill_equals_brute_force_per_sequence(rope, q_lora):
+    # packed with a block-diagonal causal mask vs the loop-level brute force
+    # run on every sequence separately (positions restart at 0)
+    from mla_inputs import make_varlen_inputs
+    cfg = tiny_cfg(rope_type=rope, q_lora_rank=q_lora)
+    lens = [3, 1, 6, 2]
+    inp, cu = make_varlen_inputs(cfg, lens, seed=31, gamma="random")
+    out, P = O.prefill_varlen(cfg, inp, cu, return_parts=True)
+    scale = O.softmax_scale(cfg)
+    r = cfg.kv_lora_rank
+    kva = inp.x[0].double().numpy() @ inp.w_kv_a.double().numpy().T
+    for b in range(len(lens)):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        ref = np.asarray(brute_prefill(cfg, _sequence_inputs(inp, lo, hi), scale))[0]
+        np.testing.assert_allclose(out[lo:hi], ref, rtol=1e-10, atol=1e-12)
+        # the first token of every sequence sits at position 0: its cached
+        # k_pe is unrotated (R_0 = I)
+        np.testing.assert_allclose(P["latent_cache"][lo, r:], kva[lo, r:],
+                                   rtol=1e-12, atol=1e-14)
+
+
+def test_varlen_prefill_single_sequence_is_prefill_and_one_token_is_v():
+    from mla_inputs import make_varlen_inputs
+    cfg = tiny_cfg()
+    inp, cu = make_varlen_inputs(cfg, [7], seed=32)
+    np.testing.assert_allclose(O.prefill_varlen(cfg, inp, cu), O.prefill(cfg, inp)[0],
+                               rtol=1e-12, atol=1e-14)
+    # a one-token sequence attends only to itself: its attention output is its
+    # own V = RMSNorm(c) W_UV, per head
+    inp, cu = make_varlen_inputs(cfg, [4, 1, 3], seed=33)
+    _, P = O.prefill_varlen(cfg, inp, cu, return_parts=True)
+    m = int(cu[1])
+    h, dn, dv, r = cfg.num_heads, cfg.qk_nope_head_dim, cfg.v_head_dim, cfg.kv_lora_rank
+    wkvb = inp.w_kv_b.double().numpy().reshape(h, dn + dv, r)
+    c_hat = P["latent_cache"][m, :r]
+    for hh in range(h):
+        np.testing.assert_allclose(P["attn"][m, hh], wkvb[hh, dn:] @ c_hat,
+                                   rtol=1e-12, atol=1e-14)
+    assert P["pos"].tolist() == [0, 1, 2, 3, 0, 0, 1, 2]
+
+
+@pytest.mark.parametrize("mistake", ["no_boundaries", "positions_not_restarted"])
+def test_planted_varlen_mistake_is_caught(monkeypatch, mistake):
+    orig = O._packed_rows
+
+    def wrong(cu, N):
+        seq, pos = orig(cu, N)
+        if mistake == "no_boundaries":
+            return np.zeros_like(seq), pos
+        return seq, np.arange(N)
+    monkeypatch.setattr(O, "_packed_rows", wrong)
+    with pytest.raises(AssertionError):
+        test_varlen_prefill_equals_brute_force_per_sequence("plain", 8)
