@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 2
+#define MLA_ABI_VERSION 3
 
 /* Exported symbols keep default visibility even when the library is built
  * with -fvisibility=hidden. */
@@ -132,9 +132,11 @@ typedef struct mla_weights {
  *   latent [B*(T_past+T), kv_lora+rope]  (mla_prefill_chunked only) the
  *                                 normalised latent rows of history and new
  *                                 tokens; kv then covers these rows
+ *   pos    [total] int32          (mla_prefill_varlen only) position of every
+ *                                 packed row within its sequence
  * Offsets are -1 for buffers a configuration does not use. */
 typedef struct mla_prefill_layout {
-  int64_t status, ssq_q, ssq_kv, q_a, ckv, q, kv, attn, total_bytes, latent;
+  int64_t status, ssq_q, ssq_kv, q_a, ckv, q, kv, attn, total_bytes, latent, pos;
 } mla_prefill_layout;
 
 /* Byte offsets of the decode intermediates inside the workspace:
@@ -256,6 +258,41 @@ MLA_API mla_status mla_prefill_chunked(const mla_config* cfg, const mla_weights*
                                        const float* rope_cos, const float* rope_sin,
                                        void* out, void* latent_cache_out, void* workspace,
                                        size_t workspace_bytes, void* stream);
+
+/* Workspace bytes mla_prefill_varlen needs; 0 if the arguments are invalid. */
+MLA_API size_t mla_prefill_varlen_workspace_size(const mla_config* cfg, int32_t n_seq,
+                                                 int32_t total, int32_t max_seqlen,
+                                                 mla_prefill_layout* layout);
+
+/*
+ * mla_prefill_varlen -- prefill of n_seq variable-length sequences packed back
+ * to back (THD layout).
+ *
+ * Megatron-LM MLA guide, 训练支持与并行策略: packed sequences are described by
+ * cumulative lengths.  Sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1;
+ * its tokens sit at positions 0, 1, ... (RoPE restarts in every sequence) and
+ * attend causally within their own sequence only.  Every other step is
+ * mla_prefill_forward's computation, row by row.
+ *
+ *   x            [total, hidden] packed tokens
+ *   cu_seqlens   DEVICE int32 [n_seq + 1], cu[0] = 0, non-decreasing,
+ *                cu[n_seq] = total, every length <= max_seqlen.  It is read on
+ *                the device only: a malformed array sets the device status word,
+ *                which mla_check_device_status reports as MLA_ERR_SHAPE; all
+ *                accesses stay clamped inside [0, total) rows.
+ *   max_seqlen   longest sequence (sizes the launch; 1 <= max_seqlen <= total)
+ *   rope_cos/sin fp32 [>= max_seqlen, rope]
+ *   out          [total, hidden]
+ *   latent_cache_out  NULL or [total, kv_lora_rank + rope], packed like x
+ *   workspace    >= mla_prefill_varlen_workspace_size bytes, 256-aligned
+ * Errors: MLA_ERR_NULL / SHAPE / ALIGN / DTYPE / WORKSPACE before any launch;
+ * MLA_ERR_UNSUPPORTED when n_seq x heads exceeds 65535 (launch grid).
+ */
+MLA_API mla_status mla_prefill_varlen(const mla_config* cfg, const mla_weights* w, const void* x,
+                                      const int32_t* cu_seqlens, int32_t n_seq, int32_t total,
+                                      int32_t max_seqlen, const float* rope_cos,
+                                      const float* rope_sin, void* out, void* latent_cache_out,
+                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes mla_decode_absorbed needs for (cfg, B, max_ctx); 0 if the
  * arguments are invalid.  Fills *layout when it is not NULL. */

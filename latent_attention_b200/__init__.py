@@ -17,6 +17,7 @@ __all__ = ["MlaError", "make_config", "mla_build_rope_tables",
            "mla_decode_workspace_size", "mla_decode_absorbed",
            "mla_check_device_status", "mla_decode_absorbed_noalloc",
            "mla_prefill_chunked_workspace_size", "mla_prefill_chunked",
+           "mla_prefill_varlen_workspace_size", "mla_prefill_varlen",
            "abi_version"]
 
 
@@ -140,6 +141,33 @@ def mla_prefill_chunked(cfg, weights, x, B, T_new, past_cache, T_past, rope_cos,
         _ptr(rope_cos, "rope_cos", True), _ptr(rope_sin, "rope_sin", True),
         _ptr(out, "out"), _ptr(latent_cache_out, "latent_cache_out", True),
         _ptr(workspace, "workspace"),
+        C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def mla_prefill_varlen_workspace_size(cfg, n_seq, total, max_seqlen):
+    c = cfg if isinstance(cfg, mla_config) else make_config(cfg)
+    lay = mla_prefill_layout()
+    n = _lib.load().mla_prefill_varlen_workspace_size(
+        C.byref(c), int(n_seq), int(total), int(max_seqlen), C.byref(lay))
+    if n == 0:
+        raise MlaError(2, "invalid configuration or sizes")
+    return n, {f: getattr(lay, f) for f, _ in lay._fields_}
+
+
+def mla_prefill_varlen(cfg, weights, x, cu_seqlens, n_seq, total, max_seqlen, rope_cos,
+                       rope_sin, out, workspace, latent_cache_out=None, stream=None):
+    """Prefill of n_seq packed sequences (rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+    of x [total, hidden]); cu_seqlens is a device int32 tensor [n_seq + 1]."""
+    import torch
+    c = cfg if isinstance(cfg, mla_config) else make_config(cfg)
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    w = _weights(weights)
+    _check(_lib.load().mla_prefill_varlen(
+        C.byref(c), C.byref(w), _ptr(x, "x"), _ptr(cu_seqlens, "cu_seqlens"), int(n_seq),
+        int(total), int(max_seqlen), _ptr(rope_cos, "rope_cos", True),
+        _ptr(rope_sin, "rope_sin", True), _ptr(out, "out"),
+        _ptr(latent_cache_out, "latent_cache_out", True), _ptr(workspace, "workspace"),
         C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
 
 

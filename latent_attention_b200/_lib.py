@@ -27,7 +27,8 @@ EXPORTED = ["mla_abi_version", "mla_status_string", "mla_last_error_detail",
             "mla_decode_absorbed", "mla_check_device_status",
             "mla_set_stage_events", "mla_kernel_launches",
             "mla_decode_absorbed_noalloc", "mla_selftest_wait_timeout",
-            "mla_prefill_chunked_workspace_size", "mla_prefill_chunked"]
+            "mla_prefill_chunked_workspace_size", "mla_prefill_chunked",
+            "mla_prefill_varlen_workspace_size", "mla_prefill_varlen"]
 
 
 class mla_config(C.Structure):
@@ -52,7 +53,7 @@ class mla_weights(C.Structure):
 class mla_prefill_layout(C.Structure):
     _fields_ = [(n, C.c_int64) for n in
                 ("status", "ssq_q", "ssq_kv", "q_a", "ckv", "q", "kv", "attn",
-                 "total_bytes", "latent")]
+                 "total_bytes", "latent", "pos")]
 
 
 class mla_decode_layout(C.Structure):
@@ -109,6 +110,12 @@ def load():
     lib.mla_prefill_chunked.restype = C.c_int
     lib.mla_prefill_chunked.argtypes = [cfgp, C.POINTER(mla_weights), vp, i32, i32, vp,
                                         i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.mla_prefill_varlen_workspace_size.restype = sz
+    lib.mla_prefill_varlen_workspace_size.argtypes = [cfgp, i32, i32, i32,
+                                                      C.POINTER(mla_prefill_layout)]
+    lib.mla_prefill_varlen.restype = C.c_int
+    lib.mla_prefill_varlen.argtypes = [cfgp, C.POINTER(mla_weights), vp, vp, i32, i32, i32,
+                                       vp, vp, vp, vp, vp, sz, vp]
     lib.mla_selftest_wait_timeout.restype = C.c_int
     lib.mla_selftest_wait_timeout.argtypes = [vp, vp]
     lib.mla_decode_absorbed_noalloc.restype = C.c_int

@@ -98,7 +98,8 @@ struct PrefillPlan {
 // Prefill workspace for B sequences of T new tokens after T_past cached ones
 // (T_past = 0: plain prefill).  Buffers over the new tokens are N = B*T rows;
 // with a cache, the full latent rows and kv cover B*(T_past + T) rows.
-void prefill_layout(const mla_config& c, int B, int T, int T_past, mla_prefill_layout* L) {
+void prefill_layout(const mla_config& c, int B, int T, int T_past, mla_prefill_layout* L,
+                    bool packed = false) {
   const int64_t N = (int64_t)B * T, Na = (int64_t)B * (T + T_past), es = elem_size(c);
   const int dq = c.qk_nope_head_dim + c.qk_rope_head_dim;
   const int w = c.kv_lora_rank + c.qk_rope_head_dim;
@@ -115,6 +116,7 @@ void prefill_layout(const mla_config& c, int B, int T, int T_past, mla_prefill_l
   L->q = take(N * c.num_heads * dq * es);
   L->kv = take(Na * c.num_heads * (c.qk_nope_head_dim + c.v_head_dim) * es);
   L->attn = take(N * c.num_heads * c.v_head_dim * es);
+  L->pos = packed ? take(N * 4) : -1;
   L->total_bytes = off;
 }
 
@@ -144,13 +146,21 @@ char* at(void* ws, int64_t off) { return off < 0 ? nullptr : static_cast<char*>(
 }  // namespace
 
 namespace {
+// Packed (THD) sequences: cu_seqlens[0..n_seq] on the device, the longest
+// sequence max_len.
+struct Packed {
+  const int32_t* cu;
+  int n_seq, max_len;
+};
+
 // Prefill of B sequences of T new tokens after T_past tokens whose latent
 // rows are in past_cache ([B, T_past, r_kv + rope]; T_past = 0: plain).
+// Packed: B = 1, T = all packed rows, T_past = 0 and `pk` describes them.
 mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* x, int32_t B,
                        int32_t T, const void* past_cache, int32_t T_past,
                        const float* rope_cos, const float* rope_sin, void* out,
                        void* latent_cache_out, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       void* stream, const Packed* pk = nullptr) {
   mla_status s = check_config(cfg);
   if (s != MLA_OK) return s;
   const mla_config& c = *cfg;
@@ -171,7 +181,7 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   if (reinterpret_cast<uintptr_t>(workspace) & 255u)
     return fail(MLA_ERR_ALIGN, "workspace is not 256-byte aligned");
   mla_prefill_layout L;
-  prefill_layout(c, B, T, T_past, &L);
+  prefill_layout(c, B, T, T_past, &L, pk != nullptr);
   if ((int64_t)workspace_bytes < L.total_bytes)
     return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
                 (long long)L.total_bytes);
@@ -199,11 +209,16 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   void* attn = at(ws, L.attn);
   void* latent = at(ws, L.latent);
   uint32_t* status = (uint32_t*)at(ws, L.status);
+  int32_t* pos = (int32_t*)at(ws, L.pos);
 
   // The status word starts at zero; every other buffer is fully written.
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   mla::stage_event(0, st);
+  if (pk) {       // per-row positions of the packed sequences (RoPE)
+    e = mla::launch_packed_positions(pk->cu, pk->n_seq, N, pk->max_len, pos, status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "packed positions");
+  }
 
   // S1: fused down-projection [x W_qa^T | x W_kva^T]; epilogue: RMS row
   // statistics, gains, RoPE on k_pe.
@@ -224,7 +239,7 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
     e1.gamma = w->g_kv_a; e1.norm_cols = r_kv; e1.ssq_out = ssq_kv; e1.ssq_ld = N;
     if (rope) {
       e1.cos = rope_cos; e1.sin = rope_sin; e1.rope_period = r_kv + dr;
-      e1.rope_start = r_kv; e1.rope_dim = dr; e1.T = T; e1.pos_offset = T_past;
+      e1.rope_start = r_kv; e1.rope_dim = dr; e1.T = T; e1.pos_offset = T_past; e1.pos = pos;
     }
     ++si;
   }
@@ -260,7 +275,7 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   eq.out = q; eq.ldo = (int64_t)h * dq; eq.ncols = h * dq;
   if (rope) {
     eq.cos = rope_cos; eq.sin = rope_sin; eq.rope_period = dq; eq.rope_start = dn;
-    eq.rope_dim = dr; eq.T = T; eq.pos_offset = T_past;
+    eq.rope_dim = dr; eq.T = T; eq.pos_offset = T_past; eq.pos = pos;
   }
   e = run_gemm(gq);
   if (e != cudaSuccess) return cuda_fail(e, "q projection");
@@ -298,6 +313,13 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   mla::AttnArgs aa{q, kv, kv_src, attn, B, T, h, dn, dr, dv, r_kv, (float)softmax_scale(c), status};
   aa.Tk = Ta;
   aa.q_off = T_past;
+  if (pk) {       // causal within each packed sequence
+    aa.B = pk->n_seq;
+    aa.T = aa.Tk = pk->max_len;
+    aa.cu_seqlens = pk->cu;
+    aa.total = N;
+  }
+  if ((int64_t)aa.B * h > 65535) return fail(MLA_ERR_UNSUPPORTED, "sequences x heads > 65535");
   e = tc_attn ? mla::tc_attention(aa, st) : mla::launch_attn_simt(c.dtype, aa, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   mla::stage_event(4, st);
@@ -415,6 +437,32 @@ mla_status mla_prefill_chunked(const mla_config* cfg, const mla_weights* w, cons
                      latent_cache_out, workspace, workspace_bytes, stream);
 }
 
+size_t mla_prefill_varlen_workspace_size(const mla_config* cfg, int32_t n_seq, int32_t total,
+                                         int32_t max_seqlen, mla_prefill_layout* layout) {
+  if (check_config(cfg) != MLA_OK || n_seq < 1 || total < 1 || max_seqlen < 1 ||
+      max_seqlen > total)
+    return 0;
+  mla_prefill_layout L;
+  prefill_layout(*cfg, 1, total, 0, &L, true);
+  if (layout) *layout = L;
+  return (size_t)L.total_bytes;
+}
+
+mla_status mla_prefill_varlen(const mla_config* cfg, const mla_weights* w, const void* x,
+                              const int32_t* cu_seqlens, int32_t n_seq, int32_t total,
+                              int32_t max_seqlen, const float* rope_cos, const float* rope_sin,
+                              void* out, void* latent_cache_out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!cu_seqlens) return fail(MLA_ERR_NULL, "cu_seqlens is NULL");
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+    return fail(MLA_ERR_ALIGN, "cu_seqlens is not 4-byte aligned");
+  if (n_seq < 1 || total < 1 || max_seqlen < 1 || max_seqlen > total)
+    return fail(MLA_ERR_SHAPE, "n_seq=%d total=%d max_seqlen=%d", n_seq, total, max_seqlen);
+  const Packed pk{cu_seqlens, n_seq, max_seqlen};
+  return run_prefill(cfg, w, x, 1, total, nullptr, 0, rope_cos, rope_sin, out, latent_cache_out,
+                     workspace, workspace_bytes, stream, &pk);
+}
+
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t B, int32_t max_ctx,
                                  mla_decode_layout* layout) {
   if (check_config(cfg) != MLA_OK || B < 1 || max_ctx < 1) return 0;
@@ -489,7 +537,7 @@ mla_status mla_check_device_status(void* workspace, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (word & mla::kStatusTimeout) return fail(MLA_ERR_DEVICE_TIMEOUT, "status word 0x%x", word);
-  if (word & mla::kStatusBadCtx) return fail(MLA_ERR_SHAPE, "cu_ctx out of range (0x%x)", word);
+  if (word & mla::kStatusBadCtx) return fail(MLA_ERR_SHAPE, "cu_ctx / cu_seqlens out of range (0x%x)", word);
   g_detail.clear();
   return MLA_OK;
 }

@@ -17,7 +17,8 @@ namespace {
 constexpr int BQ = 16, BKEY = 32, NT = 128;
 
 template <typename T>
-__global__ void __launch_bounds__(NT) attn_simt_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(NT) attn_simt_kernel(AttnArgs a_in) {
+  AttnArgs a = a_in;
   extern __shared__ float sm[];
   const int dq = a.dn + a.dr;
   float* Qs = sm;                       // [BQ][dq]
@@ -38,8 +39,16 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnArgs a) {
   const int64_t qstride = (int64_t)a.h * dq;
   const int64_t kvstride = (int64_t)a.h * (a.dn + a.dv);
   const int64_t cstride = a.r_kv + a.dr;
-  const int64_t base = (int64_t)b * a.T;        // first query row of the sequence
-  const int64_t kbase = (int64_t)b * a.Tk;      // first key row of the sequence
+  int64_t base = (int64_t)b * a.T;              // first query row of the sequence
+  int64_t kbase = (int64_t)b * a.Tk;            // first key row of the sequence
+  if (a.cu_seqlens) {   // packed: bounds clamped to [0, total)
+    const int s0 = min(max(a.cu_seqlens[b], 0), a.total);
+    const int s1 = min(max(a.cu_seqlens[b + 1], s0), a.total);
+    base = kbase = s0;
+    a.T = a.Tk = min(s1 - s0, a.T);
+    a.q_off = 0;
+  }
+  if (q0 >= a.T) return;
 
   for (int idx = tid; idx < BQ * dq; idx += NT) {
     const int i = idx / dq, d = idx % dq;

@@ -58,6 +58,8 @@ struct AttnTcParams {
   int Tk, q_off;         // keys per sequence, position of query 0
   float scale_log2;      // softmax scale * log2(e)
   int n_pairs;           // CTAs per head: ceil(T / 256)
+  const int32_t* cu;     // packed sequences (or null): rows cu[b] .. cu[b+1]-1
+  int total;             // packed row count
   __nv_bfloat16* o;      // [N, h, DV]
   uint32_t* status;
 };
@@ -80,13 +82,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int hh = blockIdx.y % p.h;
   const int b = blockIdx.y / p.h;
   const int c = p.n_pairs - 1 - blockIdx.x;          // heaviest pair first
-  const int row0 = b * p.T;                          // first query row of the sequence
-  const int krow0 = b * p.Tk;                        // first key row of the sequence
+  int row0, krow0, Tq, Tk, q_off;                    // this sequence's rows and lengths
+  if (p.cu) {   // packed: bounds clamped to [0, total) so no store leaves the buffer
+    const int s0 = min(max(p.cu[b], 0), p.total);
+    const int s1 = min(max(p.cu[b + 1], s0), p.total);
+    row0 = krow0 = s0;
+    Tq = Tk = min(s1 - s0, p.T);
+    q_off = 0;
+  } else {
+    row0 = b * p.T;
+    krow0 = b * p.Tk;
+    Tq = p.T;
+    Tk = p.Tk;
+    q_off = p.q_off;
+  }
   // tile X covers queries [q0X, q0X + 128) (positions + q_off) and key
   // blocks [0, nkvX)
   const int q0A = 256 * c, q0B = 256 * c + BQ;
-  const int nkvA = q0A < p.T ? min(p.q_off + q0A + BQ - 1, p.Tk - 1) / BKV + 1 : 0;
-  const int nkvB = q0B < p.T ? min(p.q_off + q0B + BQ - 1, p.Tk - 1) / BKV + 1 : 0;
+  if (q0A >= Tq) return;   // a shorter packed sequence: nothing for this CTA
+  const int nkvA = q0A < Tq ? min(q_off + q0A + BQ - 1, Tk - 1) / BKV + 1 : 0;
+  const int nkvB = q0B < Tq ? min(q_off + q0B + BQ - 1, Tk - 1) / BKV + 1 : 0;
   const int nkv = max(nkvA, nkvB);
 
   if (threadIdx.x == 0) {
@@ -229,7 +244,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, sr[cc]);
       tmem_wait_ld();
       // Raw scores; the scale is folded into the exp argument below (scale > 0).
-      const int kmax = min(p.q_off + qi, p.Tk - 1) - j * BKV;  // last visible key here
+      const int kmax = min(q_off + qi, Tk - 1) - j * BKV;  // last visible key here
       if (kmax < 127) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
@@ -293,7 +308,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok && my_nkv > 0 && warp_wait(&pv_done[x], (my_nkv - 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
-      const bool row_ok = qi < p.T;
+      const bool row_ok = qi < Tq;
       __nv_bfloat16* dst = p.o + ((int64_t)(row0 + qi) * p.h + hh) * DV;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
@@ -329,9 +344,10 @@ bool tc_attention_supported(const mla_config& c) {
 }
 
 cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
-  const int64_t N = (int64_t)a.B * a.T;          // query rows
   const int Tk = a.Tk > 0 ? a.Tk : a.T;
-  const int64_t Nk = (int64_t)a.B * Tk;          // key rows
+  // query and key rows of the maps (packed: all sequences' rows)
+  const int64_t N = a.cu_seqlens ? (int64_t)a.total : (int64_t)a.B * a.T;
+  const int64_t Nk = a.cu_seqlens ? (int64_t)a.total : (int64_t)a.B * Tk;
   CUtensorMap tmQ, tmKV, tmKpe;
   const uint32_t box[2] = {64, 128};
   {
@@ -361,6 +377,8 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
   p.n_pairs = (a.T + 2 * BQ - 1) / (2 * BQ);
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
   p.status = a.status;
+  p.cu = a.cu_seqlens;
+  p.total = a.total;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,

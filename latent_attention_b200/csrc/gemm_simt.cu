@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(GemmArgs a) {
     rs = rsqrtf(ss * e.rs_inv_dim + e.eps);
   }
   float ssq = 0.f;
-  const int pos = m % e.T + e.pos_offset;
+  const int pos = e.pos ? e.pos[m] : m % e.T + e.pos_offset;
   T* out = reinterpret_cast<T*>(e.out);
   for (int c = cq; c < cq + 16; ++c) {
     const int n = n0 + c;

@@ -73,7 +73,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
     for (int q = 0; q < e.ssq_parts; ++q) ss += e.ssq_in[q * e.ssq_ld + m];
     rs = rsqrtf(ss * e.rs_inv_dim + e.eps);
   }
-  const int pos = row_ok ? m % e.T + e.pos_offset : 0;
+  const int pos = row_ok ? (e.pos ? e.pos[m] : m % e.T + e.pos_offset) : 0;
   float ssq = 0.f;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out) + (int64_t)bi * p.sOut;
   const __nv_bfloat16* gamma = reinterpret_cast<const __nv_bfloat16*>(e.gamma);

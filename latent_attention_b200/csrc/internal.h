@@ -12,7 +12,7 @@ namespace mla {
 // Device status word bits (first 4 bytes of every workspace).
 enum : uint32_t {
   kStatusTimeout = 1u << 0,   // a bounded wait ran out
-  kStatusBadCtx = 1u << 1,    // decode: a cu_ctx length outside [1, max_ctx]
+  kStatusBadCtx = 1u << 1,    // a cu_ctx / cu_seqlens length outside its bounds
 };
 
 template <typename T> struct Elem;
@@ -55,6 +55,7 @@ struct EpiSeg {
   const float* sin = nullptr;
   int rope_period = 0, rope_start = 0, rope_dim = 0, T = 1;
   int pos_offset = 0;       // RoPE position = (row % T) + pos_offset
+  const int32_t* pos = nullptr;  // or, when set, the position of every row
 };
 
 // C = A B^T with A [M, K] (row stride lda) and the output columns split in up
@@ -93,6 +94,10 @@ struct AttnArgs {
   float scale;
   uint32_t* status;
   int Tk = 0, q_off = 0;
+  // Packed (THD) prefill: sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+  // of `total` rows; B is the sequence count and T the longest sequence.
+  const int32_t* cu_seqlens = nullptr;
+  int total = 0;
 };
 
 struct DecodeArgs {
@@ -129,6 +134,11 @@ cudaError_t launch_attn_simt(int dtype, const AttnArgs& a, cudaStream_t st);
 // Normalised latent rows [RMSNorm(c) | k_pe] from the gain-scaled latent
 // buffer: source row m (of N = B*T) goes to destination row
 // (m / T) * dst_T + dst_off + (m % T).
+// Packed prefill: pos[m] = m - cu_seqlens[b(m)] for the `total` packed rows;
+// malformed cu_seqlens raise kStatusBadCtx (positions stay in [0, max_len)).
+cudaError_t launch_packed_positions(const int32_t* cu_seqlens, int n_seq, int total, int max_len,
+                                    int32_t* pos, uint32_t* status, cudaStream_t st);
+
 cudaError_t launch_latent_finalize(int dtype, const void* ckv,
                                    const float* ssq_kv, int ssq_parts, int N, int r_kv,
                                    int dr, float eps, void* cache,

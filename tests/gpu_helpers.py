@@ -81,3 +81,29 @@ def run_prefill_chunked(cfg, inp, past, T_past):
     from latent_attention_b200 import mla_check_device_status
     mla_check_device_status(ws)
     return out, cache, ws, lay
+
+
+def run_prefill_varlen(cfg, inp, cu, max_len, check=True):
+    """mla_prefill_varlen on packed inputs (inp.B == 1, inp.T == total)."""
+    from latent_attention_b200 import (make_config, mla_build_rope_tables,
+                                       mla_prefill_varlen,
+                                       mla_prefill_varlen_workspace_size,
+                                       mla_check_device_status)
+    total, n_seq = inp.T, len(cu) - 1
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    c = make_config(cfg)
+    d = cfg.qk_rope_head_dim
+    cos = torch.empty(max_len, d, device="cuda")
+    sin = torch.empty_like(cos)
+    mla_build_rope_tables(c, max_len, cos, sin)
+    n, lay = mla_prefill_varlen_workspace_size(c, n_seq, total, max_len)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty(total, cfg.hidden_size, dtype=dt, device="cuda")
+    cache = torch.empty(total, cfg.kv_lora_rank + d, dtype=dt, device="cuda")
+    w = {k: (None if v is None else v.cuda()) for k, v in weights_of(inp).items()}
+    mla_prefill_varlen(c, w, inp.x.reshape(total, -1).cuda(), cu.cuda(), n_seq, total, max_len,
+                       cos, sin, out, ws, latent_cache_out=cache)
+    torch.cuda.synchronize()
+    if check:
+        mla_check_device_status(ws)
+    return out, cache, ws

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 2
+    assert lib.mla_abi_version() == 3
     for code, name in {0: b"MLA_OK", 5: b"MLA_ERR_WORKSPACE",
                        8: b"MLA_ERR_DEVICE_TIMEOUT"}.items():
         assert lib.mla_status_string(code) == name
@@ -66,6 +66,7 @@ int main(void) {
   P(mla_config, rope_theta) P(mla_config, original_max_position_embeddings)
   P(mla_config, dtype) P(mla_config, rms_eps) P(mla_config, softmax_scale)
   P(mla_weights, w_o) P(mla_decode_layout, split_tokens) P(mla_prefill_layout, latent)
+  P(mla_prefill_layout, pos)
   P(mla_decode_layout, max_splits)
   return 0;
 }
@@ -194,3 +195,30 @@ def test_chunked_prefill_validation_and_sizes(lib):
              None) == 2
     assert f(C.byref(c), C.byref(wt), p, 1, 8, _fake(0x200008), 4, p, p, p, None,
              ws, big, None) == 3
+
+
+def test_varlen_prefill_validation_and_sizes(lib):
+    from latent_attention_b200 import (make_config, mla_weights,
+                                       mla_prefill_workspace_size,
+                                       mla_prefill_varlen_workspace_size)
+    cfg = WORKLOADS["dsv3_prefill"].cfg
+    n0, l0 = mla_prefill_workspace_size(cfg, 1, 1000)
+    n1, l1 = mla_prefill_varlen_workspace_size(cfg, 7, 1000, 300)
+    assert l0["pos"] == -1 and l1["pos"] >= 0 and n1 >= n0 + 1000 * 4
+    for bad in ((0, 10, 5), (2, 0, 1), (2, 10, 11), (2, 10, 0)):
+        with pytest.raises(Exception):
+            mla_prefill_varlen_workspace_size(cfg, *bad)
+    c = make_config(cfg)
+    wt = mla_weights()
+    for i, f in enumerate(("w_q_a", "g_q_a", "w_q_b", "w_kv_a", "g_kv_a",
+                           "w_kv_b", "w_o")):
+        setattr(wt, f, 0x100000 + i * 0x1000)
+    p, ws, big = _fake(0x200000), _fake(0x1000000), C.c_size_t(1 << 40)
+    f = lib.mla_prefill_varlen
+    assert f(C.byref(c), C.byref(wt), p, None, 2, 10, 5, p, p, p, None, ws, big, None) == 1
+    assert f(C.byref(c), C.byref(wt), p, _fake(0x300002), 2, 10, 5, p, p, p, None, ws, big,
+             None) == 3
+    assert f(C.byref(c), C.byref(wt), p, p, 2, 10, 11, p, p, p, None, ws, big, None) == 2
+    assert f(C.byref(c), C.byref(wt), p, p, 0, 10, 5, p, p, p, None, ws, big, None) == 2
+    assert f(C.byref(c), C.byref(wt), p, p, 2, 10, 5, p, p, p, None, ws, C.c_size_t(64),
+             None) == 5

@@ -266,3 +266,69 @@ def test_prefill_chunked_dsv3_heads(cuda):
     out, _, _, _ = run_prefill_chunked(cfg, inp, past, T_past)
     ref = oracle.prefill_chunked(cfg, inp, past, T_past)
     assert oracle.max_rel_err(out, ref) <= TOL["bf16"]
+
+
+# --------------------------------------------------------------------------
+# Packed (THD) varlen prefill
+# --------------------------------------------------------------------------
+VARLEN = [
+    ("tiny_f32", W["tiny_f32"].cfg, [3, 1, 40, 7]),
+    ("tiny_f32_directq_norope", W["tiny_f32"].cfg.with_(q_lora_rank=0, rope_type="none"),
+     [17, 2, 33]),
+    ("bf16_dsv3dims", small_bf16(), [1, 130, 300, 257, 64]),
+    ("bf16_kimi_norope", small_bf16(rope_type="none", num_heads=3), [200, 1, 129]),
+    ("bf16_directq", small_bf16(q_lora_rank=0, rope_type="plain", num_heads=2), [256, 255, 3]),
+]
+
+
+@pytest.mark.parametrize("name,cfg,lens", VARLEN, ids=[v[0] for v in VARLEN])
+def test_prefill_varlen_small(cuda, name, cfg, lens):
+    from gpu_helpers import run_prefill_varlen
+    from mla_inputs import make_varlen_inputs
+    inp, cu = make_varlen_inputs(cfg, lens, seed=41, gamma="random")
+    out, cache, _ = run_prefill_varlen(cfg, inp, cu, max(lens))
+    ref, P = oracle.prefill_varlen(cfg, inp, cu, return_parts=True)
+    tol = TOL[cfg.dtype]
+    assert oracle.max_rel_err(out, ref) <= tol
+    assert oracle.max_rel_err(cache, P["latent_cache"]) <= tol
+
+
+def test_prefill_varlen_matches_separate_prefills(cuda):
+    """Each packed sequence gives what a prefill of that sequence alone gives."""
+    from gpu_helpers import run_prefill_varlen
+    from mla_inputs import make_varlen_inputs
+    cfg = small_bf16()
+    lens = [300, 1, 129, 512]
+    inp, cu = make_varlen_inputs(cfg, lens, seed=42)
+    out, _, _ = run_prefill_varlen(cfg, inp, cu, max(lens))
+    for b, n in enumerate(lens):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        one = type(inp)(**{**inp.__dict__, "x": inp.x[:, lo:hi], "T": n})
+        _, o1, _ = run_prefill(cfg, one, latent=False)
+        assert oracle.max_rel_err(out[lo:hi], o1[0]) <= 1e-3
+
+
+def test_prefill_varlen_dsv3_heads_sampled(cuda):
+    from gpu_helpers import run_prefill_varlen
+    from mla_inputs import make_varlen_inputs, varlen_seq_lengths
+    cfg = W["dsv3_prefill"].cfg
+    lens = varlen_seq_lengths(6, 1, 700, seed=3).tolist()
+    inp, cu = make_varlen_inputs(cfg, lens, seed=43)
+    out, _, _ = run_prefill_varlen(cfg, inp, cu, max(lens))
+    ref = oracle.prefill_varlen(cfg, inp, cu)
+    assert oracle.max_rel_err(out, ref) <= TOL["bf16"]
+
+
+def test_prefill_varlen_bad_cu_seqlens_is_flagged(cuda):
+    """A malformed cu_seqlens (decreasing, too long) is reported through the
+    status word; every access stays inside the packed rows."""
+    from latent_attention_b200 import MlaError, mla_check_device_status
+    from gpu_helpers import run_prefill_varlen
+    from mla_inputs import make_varlen_inputs
+    cfg = small_bf16()
+    inp, _ = make_varlen_inputs(cfg, [50, 50], seed=44)
+    bad = torch.tensor([0, 60, 20, 100], dtype=torch.int32)
+    _, _, ws = run_prefill_varlen(cfg, inp, bad, 60, check=False)
+    with pytest.raises(MlaError, match="SHAPE"):
+        mla_check_device_status(ws)
+    mla_check_device_status(ws)          # cleared; the context is still usable
