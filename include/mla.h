@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 3
+#define MLA_ABI_VERSION 4
 
 /* Exported symbols keep default visibility even when the library is built
  * with -fvisibility=hidden. */
@@ -108,6 +108,14 @@ typedef struct mla_config {
                                        YaRN when mscale_all_dim != 0, with
                                        m(s,a) = 0.1 a ln s + 1 for s > 1
                                        ([DSV3] __init__; [MEGATRON] 源码架构) */
+  int32_t rope_interleave;          /* 1: the projections emit each head's rope
+                                       columns as adjacent pairs (2i, 2i+1)
+                                       ("interleaved weights", [DSV3] forward);
+                                       they are de-interleaved to rotate_half
+                                       order [x0 x2 .. | x1 x3 ..] before RoPE,
+                                       so q_pe, k_pe and the latent cache come
+                                       out exactly as with the permuted weights.
+                                       0: rotate_half order already. */
 } mla_config;
 
 /* Layer weights, all [out, in] row-major in cfg->dtype. */

@@ -49,6 +49,7 @@ def make_config(cfg) -> mla_config:
     c.rope_type = ROPE_TYPES[cfg.rope_type]
     c.dtype = {"f32": MLA_F32, "bf16": MLA_BF16}[cfg.dtype]
     c.softmax_scale = float(cfg.softmax_scale or 0.0)
+    c.rope_interleave = int(bool(getattr(cfg, "rope_interleave", False)))
     return c
 
 

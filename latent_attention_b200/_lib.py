@@ -41,7 +41,7 @@ class mla_config(C.Structure):
                 ("beta_fast", C.c_double), ("beta_slow", C.c_double),
                 ("original_max_position_embeddings", C.c_int32),
                 ("dtype", C.c_int32), ("rms_eps", C.c_double),
-                ("softmax_scale", C.c_double)]
+                ("softmax_scale", C.c_double), ("rope_interleave", C.c_int32)]
 
 
 class mla_weights(C.Structure):

@@ -56,6 +56,8 @@ mla_status check_config(const mla_config* c) {
   if (!c) return fail(MLA_ERR_NULL, "cfg is NULL");
   if (c->dtype != MLA_F32 && c->dtype != MLA_BF16)
     return fail(MLA_ERR_DTYPE, "cfg->dtype=%d is not MLA_F32 or MLA_BF16", c->dtype);
+  if (c->rope_interleave != 0 && c->rope_interleave != 1)
+    return fail(MLA_ERR_SHAPE, "rope_interleave=%d is not 0 or 1", c->rope_interleave);
   const int lim = 1 << 20;
   if (c->hidden_size < 1 || c->hidden_size > lim) return fail(MLA_ERR_SHAPE, "hidden_size=%d", c->hidden_size);
   if (c->num_heads < 1 || c->num_heads > 4096) return fail(MLA_ERR_SHAPE, "num_heads=%d", c->num_heads);
@@ -240,6 +242,7 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
     if (rope) {
       e1.cos = rope_cos; e1.sin = rope_sin; e1.rope_period = r_kv + dr;
       e1.rope_start = r_kv; e1.rope_dim = dr; e1.T = T; e1.pos_offset = T_past; e1.pos = pos;
+      e1.rope_interleave = c.rope_interleave != 0;
     }
     ++si;
   }
@@ -276,6 +279,7 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   if (rope) {
     eq.cos = rope_cos; eq.sin = rope_sin; eq.rope_period = dq; eq.rope_start = dn;
     eq.rope_dim = dr; eq.T = T; eq.pos_offset = T_past; eq.pos = pos;
+    eq.rope_interleave = c.rope_interleave != 0;
   }
   e = run_gemm(gq);
   if (e != cudaSuccess) return cuda_fail(e, "q projection");

@@ -92,12 +92,17 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(GemmArgs a) {
     if (e.cos) {
       const int p = n % e.rope_period;
       if (p >= e.rope_start && p < e.rope_start + e.rope_dim) {
+        // pair (x1, x2) = columns (j, j + half) of the segment, or (2j, 2j+1)
+        // for interleaved weights; output column i is x1' (i < half) or x2'.
         const int i = p - e.rope_start;
         const int half = e.rope_dim / 2;
-        const float other = Cs[r][i < half ? c + half : c - half] * rs;
-        const float rot = i < half ? -other : other;
-        v = v * e.cos[(int64_t)pos * e.rope_dim + i] +
-            rot * e.sin[(int64_t)pos * e.rope_dim + i];
+        const int j = i < half ? i : i - half;
+        const int cb = c - i;                              // segment start in the tile
+        const float x1 = Cs[r][e.rope_interleave ? cb + 2 * j : cb + j] * rs;
+        const float x2 = Cs[r][e.rope_interleave ? cb + 2 * j + 1 : cb + j + half] * rs;
+        const float cs = e.cos[(int64_t)pos * e.rope_dim + i];
+        const float sn = e.sin[(int64_t)pos * e.rope_dim + i];
+        v = i < half ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
       }
     }
     if (e.gamma && n < e.norm_cols) v *= ld<T>(e.gamma, n);

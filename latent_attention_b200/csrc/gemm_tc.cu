@@ -100,6 +100,16 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] *= rs;
     if (e.cos && (nl % e.rope_period) == e.rope_start) {
+      if (e.rope_interleave) {   // pairs (2i, 2i+1) -> rotate_half order (i, i + 32)
+        float u[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) u[i] = v[i];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          v[i] = u[2 * i];
+          v[i + 32] = u[2 * i + 1];
+        }
+      }
       // rotate_half RoPE on a 64-wide rope segment: pairs (i, i + 32).
       const float4* cs = reinterpret_cast<const float4*>(e.cos + (int64_t)pos * 64);
       const float4* sn = reinterpret_cast<const float4*>(e.sin + (int64_t)pos * 64);

@@ -56,6 +56,7 @@ struct EpiSeg {
   int rope_period = 0, rope_start = 0, rope_dim = 0, T = 1;
   int pos_offset = 0;       // RoPE position = (row % T) + pos_offset
   const int32_t* pos = nullptr;  // or, when set, the position of every row
+  bool rope_interleave = false;  // rope columns arrive as pairs (2i, 2i+1)
 };
 
 // C = A B^T with A [M, K] (row stride lda) and the output columns split in up

@@ -33,6 +33,7 @@ class MlaConfig:
     rms_eps: float = 1e-6
     softmax_scale: Optional[float] = None   # None: derived from head dim + YaRN
     dtype: str = "bf16"                     # "bf16" | "f32"
+    rope_interleave: bool = False           # rope columns as adjacent pairs
 
     @property
     def qk_head_dim(self) -> int:

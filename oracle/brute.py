@@ -60,6 +60,7 @@ def brute_prefill(cfg, inp, scale):
     dn, dr, dv = cfg.qk_nope_head_dim, cfg.qk_rope_head_dim, cfg.v_head_dim
     dq = dn + dr
     r_kv = cfg.kv_lora_rank
+    assert not getattr(cfg, "rope_interleave", False)
     rotate = cfg.rope_type == "plain"
     X = _tolist(inp.x)
     Wkva, Wkvb, Wo = _tolist(inp.w_kv_a), _tolist(inp.w_kv_b), _tolist(inp.w_o)

@@ -151,6 +151,16 @@ def apply_rope(x, cos, sin):
     return x * cos + rotate_half(x) * sin
 
 
+def _rope_columns(cfg, x):
+    """[DSV3] forward: with ``rope_interleave`` the projections emit the rope
+    columns as adjacent pairs (2i, 2i+1), and apply_rotary_pos_emb_interleave
+    first brings them to rotate_half order [x0, x2, .., x(d-2), x1, x3, ..]
+    (pair i becomes columns (i, i + d/2)) and then rotates as usual."""
+    if not getattr(cfg, "rope_interleave", False):
+        return x
+    return np.concatenate([x[..., 0::2], x[..., 1::2]], axis=-1)
+
+
 # ---------------------------------------------------------------------------
 # RMSNorm (S2)
 # ---------------------------------------------------------------------------
@@ -231,6 +241,7 @@ def prefill(cfg, inp, rows: Optional[Sequence[int]] = None,
 
     # Step 4: RoPE at position t (0-based within the batch row).
     if cfg.rope_type != "none":
+        q_pe, kpe = _rope_columns(cfg, q_pe), _rope_columns(cfg, kpe)
         cos, sin = rope_tables(cfg, T)
         kpe = apply_rope(kpe, cos[None, :, :], sin[None, :, :])
         q_pe = apply_rope(q_pe, cos[rows][None, :, None, :],
@@ -307,6 +318,7 @@ def prefill_chunked(cfg, inp, past_cache, T_past: int,
     q = q.reshape(B, Tn, h, dq)
     q_nope, q_pe = q[..., :dn], q[..., dn:]
     if cfg.rope_type != "none":
+        q_pe, kpe = _rope_columns(cfg, q_pe), _rope_columns(cfg, kpe)
         cos, sin = rope_tables(cfg, Ta)
         cn, sn = cos[T_past:Ta], sin[T_past:Ta]
         kpe = apply_rope(kpe, cn[None], sn[None])
@@ -375,6 +387,7 @@ def prefill_varlen(cfg, inp, cu_seqlens, return_parts: bool = False):
     q = q.reshape(N, h, dq)
     q_nope, q_pe = q[..., :dn], q[..., dn:]
     if cfg.rope_type != "none":
+        q_pe, kpe = _rope_columns(cfg, q_pe), _rope_columns(cfg, kpe)
         cos, sin = rope_tables(cfg, int(pos.max()) + 1 if N else 1)
         kpe = apply_rope(kpe, cos[pos], sin[pos])
         q_pe = apply_rope(q_pe, cos[pos][:, None, :], sin[pos][:, None, :])

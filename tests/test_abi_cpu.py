@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 3
+    assert lib.mla_abi_version() == 4
     for code, name in {0: b"MLA_OK", 5: b"MLA_ERR_WORKSPACE",
                        8: b"MLA_ERR_DEVICE_TIMEOUT"}.items():
         assert lib.mla_status_string(code) == name
@@ -66,7 +66,7 @@ int main(void) {
   P(mla_config, rope_theta) P(mla_config, original_max_position_embeddings)
   P(mla_config, dtype) P(mla_config, rms_eps) P(mla_config, softmax_scale)
   P(mla_weights, w_o) P(mla_decode_layout, split_tokens) P(mla_prefill_layout, latent)
-  P(mla_prefill_layout, pos)
+  P(mla_prefill_layout, pos) P(mla_config, rope_interleave)
   P(mla_decode_layout, max_splits)
   return 0;
 }

@@ -332,3 +332,39 @@ def test_prefill_varlen_bad_cu_seqlens_is_flagged(cuda):
     with pytest.raises(MlaError, match="SHAPE"):
         mla_check_device_status(ws)
     mla_check_device_status(ws)          # cleared; the context is still usable
+
+
+# --------------------------------------------------------------------------
+# rope_interleave weights
+# --------------------------------------------------------------------------
+INTERLEAVE = [
+    ("tiny_f32", W["tiny_f32"].cfg.with_(rope_interleave=True), 2, 37),
+    ("bf16_dsv3dims_yarn", small_bf16(rope_interleave=True), 2, 300),
+    ("bf16_directq", small_bf16(q_lora_rank=0, rope_type="plain", num_heads=2,
+                                rope_interleave=True), 1, 129),
+]
+
+
+@pytest.mark.parametrize("name,cfg,B,T", INTERLEAVE, ids=[c[0] for c in INTERLEAVE])
+def test_prefill_rope_interleave(cuda, name, cfg, B, T):
+    inp = make_prefill_inputs(cfg, B, T, seed=52, gamma="random")
+    _, out, cache = run_prefill(cfg, inp)
+    ref, P = oracle.prefill(cfg, inp, return_parts=True)
+    tol = TOL[cfg.dtype]
+    assert oracle.max_rel_err(out, ref) <= tol
+    assert oracle.max_rel_err(cache.view(B, T, -1), P["latent_cache"]) <= tol
+
+
+def test_varlen_and_chunked_with_rope_interleave(cuda):
+    from gpu_helpers import run_prefill_varlen, run_prefill_chunked
+    from mla_inputs import make_varlen_inputs
+    cfg = small_bf16(rope_interleave=True)
+    inp, cu = make_varlen_inputs(cfg, [70, 1, 200], seed=53)
+    out, _, _ = run_prefill_varlen(cfg, inp, cu, 200)
+    assert oracle.max_rel_err(out, oracle.prefill_varlen(cfg, inp, cu)) <= TOL["bf16"]
+    new = make_prefill_inputs(cfg, 1, 90, seed=54)
+    g = torch.Generator().manual_seed(55)
+    past = torch.randn(1, 150, cfg.kv_lora_rank + cfg.qk_rope_head_dim,
+                       generator=g).to(torch.bfloat16)
+    out_c, _, _, _ = run_prefill_chunked(cfg, new, past, 150)
+    assert oracle.max_rel_err(out_c, oracle.prefill_chunked(cfg, new, past, 150)) <= TOL["bf16"]

@@ -459,3 +459,44 @@ def test_planted_varlen_mistake_is_caught(monkeypatch, mistake):
     monkeypatch.setattr(O, "_packed_rows", wrong)
     with pytest.raises(AssertionError):
         test_varlen_prefill_equals_brute_force_per_sequence("plain", 8)
+
+
+# --------------------------------------------------------------------------
+# rope_interleave (CSDN DeepseekV3Attention forward: "interleaved weights")
+# --------------------------------------------------------------------------
+def _deinterleave_weights(cfg, inp):
+    """The same layer with standard weights: the rope output rows of the q and
+    kv_a projections permuted from pair order (2i, 2i+1) to rotate_half order."""
+    dr, dn, r = cfg.qk_rope_head_dim, cfg.qk_nope_head_dim, cfg.kv_lora_rank
+    perm = list(range(0, dr, 2)) + list(range(1, dr, 2))
+    dq = dn + dr
+    q_rows = [hh * dq + (i if i < dn else dn + perm[i - dn])
+              for hh in range(cfg.num_heads) for i in range(dq)]
+    kv_rows = list(range(r)) + [r + p for p in perm]
+    kw = dict(w_kv_a=inp.w_kv_a[kv_rows])
+    if cfg.q_lora_rank > 0:
+        kw["w_q_b"] = inp.w_q_b[q_rows]
+    else:
+        kw["w_q"] = inp.w_q[q_rows]
+    return type(inp)(**{**inp.__dict__, **kw})
+
+
+@pytest.mark.parametrize("q_lora", [8, 0])
+def test_rope_interleave_equals_permuted_weights(q_lora):
+    # brute force with the permuted (standard) weights vs the oracle with the
+    # interleaved flag on the original weights: outputs and cached k_pe agree
+    cfg_i = tiny_cfg(q_lora_rank=q_lora, rope_interleave=True)
+    cfg_p = cfg_i.with_(rope_interleave=False)
+    inp = make_prefill_inputs(cfg_i, 2, 5, seed=51, gamma="random", w_std=0.4)
+    out_i, P = O.prefill(cfg_i, inp, return_parts=True)
+    perm_inp = _deinterleave_weights(cfg_i, inp)
+    ref = np.asarray(brute_prefill(cfg_p, perm_inp, O.softmax_scale(cfg_p)))
+    np.testing.assert_allclose(out_i, ref, rtol=1e-10, atol=1e-12)
+    _, Pp = O.prefill(cfg_p, perm_inp, return_parts=True)
+    np.testing.assert_allclose(P["latent_cache"], Pp["latent_cache"], rtol=1e-12, atol=1e-14)
+
+
+def test_planted_interleave_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "_rope_columns", lambda cfg, x: x)
+    with pytest.raises(AssertionError):
+        test_rope_interleave_equals_permuted_weights(8)
