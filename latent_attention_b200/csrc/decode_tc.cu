@@ -28,11 +28,12 @@
 // chunks ahead of the PV product (three chunk stages, three score slots), so
 // the exchange and softmax of chunk j overlap the tensor work of j+1 and j+2.
 // P_j (bf16 pairs) is written over the first half of S_j's TMEM slot.
-// Warp roles (320 threads per CTA):
+// Warp roles (448 threads per CTA):
 //   warp 0     TMA: Q share once, chunk ring (3 stages), L2 prefetch ahead
 //   warp 1     TMEM allocation, MMA issue (S_j, then O += P_{j-2} C_{j-2})
 //   warps 2, 3, 8, 9  score exchange (fp16 partial to the peer)
-//   warps 4-7  softmax (thread = head), P into TMEM, epilogue
+//   warps 4-7, 10-13  two softmax groups taking alternate chunks (thread =
+//              head), P into TMEM; group 0 also writes the epilogue
 // All waits are bounded; a timeout sets the device status word.
 #include <cfloat>
 #include <cuda_fp16.h>
@@ -58,7 +59,7 @@ constexpr int STAGE = MAX_ATOMS * CBOX;                  // 40 KB
 constexpr int XBUF = 128 * NT * 2;                       // exchange: 128 x 64 fp16
 constexpr int OFF_X = OFF_C + NSTAGE * STAGE;            // peer partials received (x2)
 constexpr int SMEM_BYTES = OFF_X + 2 * XBUF + 1024;
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 448;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
@@ -130,7 +131,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full, qpe_full, c_full[NSTAGE], c_empty[NSTAGE],
-      s_full[NSTAGE], s_free[NSTAGE], p_full[NSTAGE], pv_done[2], o_done, x_full[2], x_empty[2];
+      s_full[NSTAGE], s_free[NSTAGE], p_full[NSTAGE], pv_done[2], o_done, x_full[2], x_empty[2],
+      ref_ready[2], fin;
+  __shared__ float m_hand[2][128];          // reference max after chunk j, slot j % 2
+  __shared__ float m_fin[128], l_fin[128];  // softmax group 1's final reference and sum
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -173,7 +177,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&x_full[s], 1);    // one local arrive.expect_tx + the peer's st.async bytes
       mbar_init(&x_empty[s], 4);   // one arrive per softmax warp of the peer
+      mbar_init(&ref_ready[s], 4); // a softmax group published chunk j's reference
     }
+    mbar_init(&fin, 4);            // softmax group 1 published its final sum
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -188,6 +194,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // exchange warps 2, 3, 8, 9 and softmax warps 4..7 each cover TMEM lane
   // quarter (warp & 3), i.e. heads 32 * (warp & 3) .. + 31.
   const bool xwg = warp == 2 || warp == 3 || warp == 8 || warp == 9;
+  // softmax groups: warps 4..7 (group 0) and 10..13 (group 1)
+  const int sm_wg = (warp >= 4 && warp < 8) ? 0 : (warp >= 10 ? 1 : -1);
 
   if (warp == 0) {
     if (elect_one()) {
@@ -217,38 +225,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_Q));
       bool ok = mbar_wait(&q_full, 0, abort_v, p.status);
       if (ok && rope) ok = mbar_wait(&qpe_full, 0, abort_v, p.status);
-      for (int j = 0; ok && j < nch + 2; ++j) {
-        if (j < nch) {   // S_j into slot j % 3
-          const int st = j % NSTAGE;
-          if (!mbar_wait(&c_full[st], (j / NSTAGE) & 1, abort_v, p.status)) break;
-          // the slot's previous scores S_{j-3} were read by the exchange warps;
-          // its P_{j-3} was consumed by PV_{j-3}, issued before this point
-          if (j >= NSTAGE &&
-              !mbar_wait(&s_free[st], ((j - NSTAGE) / NSTAGE) & 1, abort_v, p.status))
-            break;
-          tc_fence_after();
-          const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
-          issue_scores<QATOMS>(tbase + TM_S + st * NT, dq, dc);
-          if (rope) {
+      // Issue S_js and O += P_jp C_jp in whichever order their inputs become
+      // ready.  S_js reuses the slot of S_{js-3}/P_{js-3}, so it waits for
+      // PV_{js-3} to be issued (js < jp + 3); PV_jp follows S_jp.
+      int js = 0, jp = 0;
+      const uint64_t t_start = globaltimer();
+      uint32_t idle = 0;
+      while (ok && jp < nch) {
+        bool progress = false;
+        if (js < nch && js < jp + NSTAGE) {
+          const int st = js % NSTAGE;
+          if (mbar_test(&c_full[st], (js / NSTAGE) & 1) &&
+              (js < NSTAGE || mbar_test(&s_free[st], ((js - NSTAGE) / NSTAGE) & 1))) {
+            tc_fence_after();
+            const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
+            issue_scores<QATOMS>(tbase + TM_S + st * NT, dq, dc);
+            if (rope) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)   // A = rope query from TMEM, 8 columns per K step
-              mma_bf16_ts(tbase + TM_S + st * NT, tbase + TM_QPE + k * 8,
-                          dc + (uint64_t)((QATOMS * CBOX + k * 32) >> 4), IDESC_S, 1);
+              for (int k = 0; k < 4; ++k)   // A = rope query from TMEM, 8 columns per K step
+                mma_bf16_ts(tbase + TM_S + st * NT, tbase + TM_QPE + k * 8,
+                            dc + (uint64_t)((QATOMS * CBOX + k * 32) >> 4), IDESC_S, 1);
+            }
+            mma_commit(&s_full[st]);
+            ++js;
+            progress = true;
           }
-          mma_commit(&s_full[st]);
         }
-        if (j >= 2) {    // O += P_{j-2} C_{j-2}
-          const int jj = j - 2, st = jj % NSTAGE;
-          if (!mbar_wait(&p_full[st], (jj / NSTAGE) & 1, abort_v, p.status)) break;
-          tc_fence_after();
-          const uint64_t dv = desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE), CBOX);
+        if (jp < js) {
+          const int st = jp % NSTAGE;
+          if (mbar_test(&p_full[st], (jp / NSTAGE) & 1)) {
+            tc_fence_after();
+            const uint64_t dv = desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE), CBOX);
 #pragma unroll
-          for (int k = 0; k < NT / 16; ++k)
-            mma_bf16_ts(tbase + TM_O, tbase + TM_S + st * NT + k * 8,
-                        dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (jj | k) != 0);
-          mma_commit(&c_empty[st]);
-          mma_commit(&pv_done[jj & 1]);
-          if (jj == nch - 1) mma_commit(&o_done);
+            for (int k = 0; k < NT / 16; ++k)
+              mma_bf16_ts(tbase + TM_O, tbase + TM_S + st * NT + k * 8,
+                          dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (jp | k) != 0);
+            mma_commit(&c_empty[st]);
+            mma_commit(&pv_done[jp & 1]);
+            if (jp == nch - 1) mma_commit(&o_done);
+            ++jp;
+            progress = true;
+          }
+        }
+        if (progress) {
+          idle = 0;
+        } else if ((++idle & 63u) == 0) {   // bounded like every other wait
+          if (*abort_v) {
+            ok = false;
+          } else if (globaltimer() - t_start > kWaitNs) {
+            *abort_v = 1;
+            atomicOr(p.status, kStatusTimeout);
+            ok = false;
+          }
         }
       }
     }
@@ -283,14 +311,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         st_async_v4(px + r * 128 + ((c ^ (r & 7)) << 4), h[4 * c], h[4 * c + 1], h[4 * c + 2],
                     h[4 * c + 3], px_full);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------- softmax (thread = head) + epilogue
+  } else if (sm_wg >= 0) {
+    // ---------------- softmax (thread = head): warpgroup g takes chunks
+    // g, g + 2, ...  The reference max of every row passes from one group to
+    // the other through shared memory (chunk j needs chunk j-1's); each group
+    // keeps the row sum of its own chunks, relative to its last reference.
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int head = h0 + r;
     const bool head_ok = head < p.h;
-    if (rope) {      // rope part of this head's query into TMEM (A operand layout)
+    if (rope && sm_wg == 0) {   // rope part of this head's query into TMEM (A operand layout)
       uint32_t q[32];
       const uint4* src = reinterpret_cast<const uint4*>(p.q_pe + ((int64_t)b * p.h + head) * DR);
 #pragma unroll
@@ -309,7 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nch; ++j) {
+    for (int j = sm_wg; j < nch; j += 2) {
       const int st = j % NSTAGE, xs = j & 1;
       if (!warp_wait(&s_full[st], (j / NSTAGE) & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
@@ -322,10 +353,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // S_j = own fp32 partial + the peer's fp16 partial
       const uint32_t sx = smem_u32(smem + OFF_X + xs * XBUF);
       float s[NT];
+      uint32_t dep = 0;               // depends on every word loaded below
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t t[4];
         ld_shared_v4u(sx + r * 128 + ((c ^ (r & 7)) << 4), t[0], t[1], t[2], t[3]);
+        dep ^= (t[0] ^ t[1]) ^ (t[2] ^ t[3]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = 8 * c + 2 * e;
@@ -337,6 +370,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           s[i + 1] = s1;
         }
       }
+      // The receive buffer of chunk j may be refilled by the peer: the loads
+      // from it have completed, since `dep` (an input below) needs them all.
+      asm volatile("" ::"r"(dep));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(map_peer(smem_u32(&x_empty[xs]), peer));
       // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
       const int lo = j * NT - (chunk_base(n, t0, j) - t0);
       const int hi = tcount - (chunk_base(n, t0, j) - t0);
@@ -349,12 +387,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int i = 0; i < NT; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], s[i], s[i + 1]);
-      const float mx = fmaxf(m_ref, max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * p.scale_log2);
-      const bool grow = mx > m_ref + kRescaleLog2;
-      const float alpha = grow ? ex2(m_ref - mx) : 1.f;
-      if (grow) {
-        l *= alpha;
-        m_ref = mx;
+      const float cmax = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+      // reference of chunk j-1, left by the other group
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        if (!warp_wait(&ref_ready[xs ^ 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        m_prev = m_hand[xs ^ 1][r];
+      }
+      // lazy rescaling: a new reference only when the max grew by > 2^8
+      const bool grow = cmax > m_prev + kRescaleLog2;     // always at j = 0
+      const float m_new = grow ? cmax : m_prev;
+      m_hand[xs][r] = m_new;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ref_ready[xs]);
+      if (m_new != m_ref) {          // this group's sum, moved to the new reference
+        l *= ex2(m_ref - m_new);
+        m_ref = m_new;
       }
       const float neg_m = -m_ref;
       float ls[8];
@@ -371,8 +422,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         w[e] = pack_bf16(p0, p1);
       }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      // A rescale of O needs every earlier PV finished; PV_{j-1} is the last.
+      // O holds the sum through chunk j-1 at reference m_prev: rescale it
+      // when this chunk moved the reference (PV_{j-1} must be complete).
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        const float alpha = ex2(m_prev - m_new);
         if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
           ok = false;
           break;
@@ -395,14 +448,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&p_full[st]);
-        // The receive buffer of chunk j is consumed: every value loaded from
-        // it fed P_j, whose TMEM store has completed.
-        mbar_arrive_remote_relaxed(map_peer(smem_u32(&x_empty[xs]), peer));
-      }
+      if (lane == 0) mbar_arrive(&p_full[st]);
     }
-    if (ok && warp_wait(&o_done, 0, abort_v, p.status)) {
+    // Row sum of the split: both groups' sums at the last chunk's reference
+    // (references never decrease, so that is the larger of the two).
+    if (sm_wg == 1) {
+      m_fin[r] = m_ref;
+      l_fin[r] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&fin);
+    } else if (ok && warp_wait(&fin, 0, abort_v, p.status) &&
+               warp_wait(&o_done, 0, abort_v, p.status)) {
+      const float m1 = m_fin[r], l1 = l_fin[r];
+      const float m_last = fmaxf(m_ref, m1);
+      const float l_tot = l * ex2(m_ref - m_last) + (l1 > 0.f ? l1 * ex2(m1 - m_last) : 0.f);
+      m_ref = m_last;
+      l = l_tot;
       tc_fence_after();
       const int64_t part = ((int64_t)b * p.max_splits + sp) * p.h + head;
       const float inv = 1.f / l;
