@@ -186,6 +186,23 @@ def oracle_prefill_sample(cfg, inp, rows):
     return dt, done
 
 
+def rank_seeds(rank):
+    """Seeds of one rank's own synthetic inputs: every replica draws
+    different data of the same shapes."""
+    return {"prefill": 1000 * rank, "ctx": rank, "decode": 1000 * rank + 1}
+
+
+def max_over_ranks(values, world, device):
+    """Per-rank timings -> their maximum over all ranks (every rank gets it).
+    The same collective runs on every rank, in the same order."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def cpu_threads():
     try:
         import torch
@@ -282,15 +299,16 @@ def main():
     wl, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
     cfg, cfgd = wl.cfg, wd.cfg
     B, T = wl.batch, wl.seq_len
-    inp = make_prefill_inputs(cfg, B, T, seed=1000 * rank)
+    seeds = rank_seeds(rank)
+    inp = make_prefill_inputs(cfg, B, T, seed=seeds["prefill"])
     weights = {k: getattr(inp, k) for k in ("w_q_a", "g_q_a", "w_q_b", "w_q",
                                               "w_kv_a", "g_kv_a", "w_kv_b", "w_o")}
     pre = MlaPrefill(cfg, weights, B, T, device=dev)
     x = inp.x.to(dev)
     out = torch.empty(B, T, cfg.hidden_size, dtype=torch.bfloat16, device=dev)
 
-    ctx = decode_context_lengths(wd.batch, wd.ctx_min, wd.ctx_max, seed=rank)
-    di = make_decode_inputs(cfgd, wd.batch, ctx, seed=1000 * rank + 1)
+    ctx = decode_context_lengths(wd.batch, wd.ctx_min, wd.ctx_max, seed=seeds["ctx"])
+    di = make_decode_inputs(cfgd, wd.batch, ctx, seed=seeds["decode"])
     dec = MlaDecode(cfgd, wd.batch, wd.ctx_max, device=dev)
     qn, qp = di.q_nope.to(dev), di.q_pe.to(dev)
     wkvb, cache, cu = di.w_kv_b.to(dev), di.cache.to(dev), di.cu_ctx.to(dev)
@@ -358,10 +376,7 @@ def main():
             for k, n in enumerate(STAGES_P)}
     st_d = {n: sum(e[k].elapsed_time(e[k + 1]) for e in ev_d) / K
             for k, n in enumerate(STAGES_D)}
-    t = torch.tensor([step_ms, pre_ms, dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, pre_ms, dec_ms = t.tolist()
+    step_ms, pre_ms, dec_ms = max_over_ranks([step_ms, pre_ms, dec_ms], world, dev)
 
     # ---- end to end through the public API with host buffers -------------
     # Every step copies its input from pinned host memory, runs the prefill
@@ -409,7 +424,7 @@ def main():
     e2e_t0, e2e_t1 = mk(), mk()
     pipelined(Wm, K, e2e_t0, e2e_t1)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e2e_t0.elapsed_time(e2e_t1)], dtype=torch.float64, device=dev)
+    e2e_ms = e2e_t0.elapsed_time(e2e_t1)
     # serial form: one step at a time on the default stream
     ser_ev = [(mk(), mk()) for _ in range(K)]
     for i in range(Wm + K):
@@ -421,13 +436,8 @@ def main():
         if i >= Wm:
             ser_ev[i - Wm][1].record()
     torch.cuda.synchronize()
-    ser_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ser_ev)], dtype=torch.float64,
-                          device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        dist.all_reduce(ser_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
-    ser_ms = float(ser_ms.item())
+    ser_ms = sum(a.elapsed_time(b) for a, b in ser_ev)
+    e2e_ms, ser_ms = max_over_ranks([e2e_ms, ser_ms], world, dev)
 
     fl = prefill_stage_flops(cfg, B, T)
     pflops = sum(fl.values())

@@ -1,0 +1,74 @@
+"""The N > 1 host path of bench.py on CPU: two gloo ranks on 127.0.0.1.
+
+The hot path partitions by sequence, so ranks are independent replicas; the
+only collectives are the barrier and the max-over-ranks reduction of the
+timings.  These tests run that logic with world_size 2 and no GPU.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+from conftest import ROOT
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    from datetime import timedelta
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=60))
+    try:
+        # rank r times (1 + r, 10 - r, 5): every rank must see the maxima
+        got = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 5.0], world, "cpu")
+        dist.barrier()
+        q.put((rank, got, bench.rank_seeds(rank)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_seeds_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in procs:
+        rank, got, seeds = q.get(timeout=120)
+        res[rank] = (got, seeds)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0][0] == res[1][0] == [2.0, 10.0, 5.0]
+    # each replica draws its own data
+    for k in res[0][1]:
+        assert res[0][1][k] != res[1][1][k], k
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl",
+                          "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=120, env=env, cwd=ROOT)
+    assert out.returncode == 0
+    assert out.stdout.strip() == ""
+
+
+def test_max_over_ranks_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks([3.5, 1.0], 1, "cpu") == [3.5, 1.0]
