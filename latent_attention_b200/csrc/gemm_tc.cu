@@ -31,7 +31,11 @@ constexpr int BM = 128, BN = kTcTileN, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+// Output staging for TMA stores: per epilogue warp two 32-row x 64-column
+// bf16 boxes (4 KB each), 128-byte swizzled.
+constexpr int OUT_BOX = 32 * 64 * 2;
+constexpr int OFF_OUT = STAGES * STAGE_BYTES;
+constexpr int SMEM_BYTES = OFF_OUT + 4 * 2 * OUT_BOX + 1024;
 constexpr int NTHREADS = 192;
 constexpr uint32_t IDESC = idesc_bf16(BM, BN);
 constexpr uint32_t IDESC_BMN = idesc_bf16(BM, BN, 0, 1);
@@ -47,6 +51,7 @@ struct TcGemmParams {
   int total_tiles;
   int a_batch_inner, b_mn;
   int64_t sOut;
+  int tma_store;          // outputs written by TMA stores (non-batched bf16)
   EpiSeg seg[2];
   uint32_t* status;
 };
@@ -64,7 +69,8 @@ __device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& b
 
 // Epilogue of one 128 x BN tile; this thread owns output row m0 + row.
 __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSeg& e, int bi,
-                                              int m0, int n0, int row, uint32_t taddr) {
+                                              int m0, int n0, int row, uint32_t taddr,
+                                              const CUtensorMap* tmO, uint32_t stg, int& gidx) {
   const int m = m0 + row;
   const bool row_ok = m < p.M;
   float rs = 1.f;
@@ -134,7 +140,28 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
       for (int i = 0; i < 64; ++i)
         if (i < lim) v[i] *= __bfloat162float(gamma[nl + i]);
     }
-    if (row_ok) {
+    if (p.tma_store) {
+      // this warp's 32 rows x 64 columns through shared memory, one TMA store
+      const int lane = row & 31;
+      const uint32_t sb = stg + (gidx & 1) * OUT_BOX;
+      if (gidx >= 2) {            // the store issued from this box two groups ago
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(sb + lane * 128 + ((c ^ (lane & 7)) << 4),
+                     pack_bf16(v[8 * c], v[8 * c + 1]), pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                     pack_bf16(v[8 * c + 4], v[8 * c + 5]),
+                     pack_bf16(v[8 * c + 6], v[8 * c + 7]));
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0 && m0 + (row & ~31) < p.M) {   // boxes wholly below M: nothing to write
+        tma_store_2d(tmO, sb, nl, m0 + (row & ~31));
+        bulk_commit_group();
+      }
+      ++gidx;
+    } else if (row_ok) {
       __nv_bfloat16* dst = out + (int64_t)m * e.ldo + nl;
       const int lim = e.ncols - nl;
 #pragma unroll
@@ -152,6 +179,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmO0,
+                   const __grid_constant__ CUtensorMap tmO1,
                    const __grid_constant__ TcGemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2];
@@ -256,6 +285,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
+    const uint32_t stg = smem_u32(smem + OFF_OUT + quad * 2 * OUT_BOX);
+    int gidx = 0;
     int local = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
@@ -265,11 +296,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int bi, s, m0, n0;
       tile_coords(p, t, bi, s, m0, n0);
       epilogue_tile(p, p.seg[s], bi, m0, n0, row,
-                    tbase + ((uint32_t)(quad * 32) << 16) + buf * BN);
+                    tbase + ((uint32_t)(quad * 32) << 16) + buf * BN, s ? &tmO1 : &tmO0, stg,
+                    gidx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
     }
+    if (p.tma_store && lane == 0) bulk_wait_group<0>();   // stores done before exit
   }
 done:
   __syncwarp();
@@ -360,6 +393,23 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
     tmB[1] = tmB[0];
     p.tiles_n[1] = 0;
   }
+  // Outputs of a non-batched GEMM go out by TMA stores: boxes of 32 rows x
+  // 64 columns, 128-byte swizzled, clipped at the tensor's edges.
+  CUtensorMap tmO[2];
+  p.tma_store = a.batch == 1;
+  for (int s = 0; s < a.nseg && p.tma_store; ++s) {
+    const EpiSeg& e = a.seg[s];
+    if (!aligned16(e.out) || (e.ldo * 2) % 16 != 0) {
+      p.tma_store = 0;
+      break;
+    }
+    const uint64_t dims[2] = {(uint64_t)e.ncols, (uint64_t)a.M};
+    const uint64_t strides[1] = {(uint64_t)e.ldo * 2};
+    const uint32_t box[2] = {64, 32};
+    if (!encode_tmap(&tmO[s], e.out, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  if (!p.tma_store || a.nseg == 1) tmO[1] = p.tma_store ? tmO[0] : tmA;
+  if (!p.tma_store) tmO[0] = tmA;
   p.total_tiles = p.per_batch * a.batch;
   p.a_batch_inner = a.a_batch_inner;
   p.b_mn = a.b_mn;
@@ -373,7 +423,7 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
     attr = true;
   }
   const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
-  gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmA, tmB[0], tmB[1], p);
+  gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);
   count_launches();
   return cudaGetLastError();
 }
