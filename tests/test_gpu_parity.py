@@ -65,6 +65,7 @@ PREFILL_SMALL = [
      1, 257, "ones"),
     ("bf16_kimi_norope", small_bf16(rope_type="none", num_heads=3), 1, 200, "ones"),
     ("bf16_T1", small_bf16(), 2, 1, "ones"),
+    ("bf16_96_heads", small_bf16(num_heads=96, hidden_size=256), 1, 130, "random"),
 ]
 
 
@@ -145,6 +146,10 @@ DECODE_SMALL = [
     ("tiny_f32", W["tiny_f32"].cfg, [1, 7, 64, 130], 200),
     ("bf16_dsv3dims", small_bf16(), [1, 5, 300, 2049, 77], 4096),
     ("bf16_dsv3_heads", W["dsv3_decode"].cfg, [1, 1000, 33], 1024),
+    # chunk (64-token) and split (4096-token) edges, several splits per sequence
+    ("bf16_dsv3_heads_edges", W["dsv3_decode"].cfg, [63, 64, 65, 4096, 4097, 8192], 8192),
+    # 96 heads (Kimi-K3 MLA): a partial 128-head tile
+    ("bf16_96_heads", W["dsv3_decode"].cfg.with_(num_heads=96), [1, 128, 4100], 8192),
 ]
 
 
