@@ -96,59 +96,79 @@ def load_traffic():
 # Clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle-reason samples every 20 ms with timestamps.
+    Started before the warm-up and running by the time the timed region
+    begins; only samples inside the timed window are summarised (the nearest
+    ones, flagged, when the window is shorter than the sampling period)."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index):
         self.idx = gpu_index
         self.proc = None
         self.lines = []
+        self.window = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 3.0:   # sampler live
+                time.sleep(0.01)
         except (OSError, ValueError):
             self.proc = None
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t_begin, t_end):
+        self.window = (t_begin, t_end)
 
     def stop(self):
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        time.sleep(0.25)
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        for l in self.lines:
-            p = [x.strip() for x in l.split(",")]
-            if len(p) < 8:
+        rows = []
+        for t_read, l in self.lines:
+            q = [x.strip() for x in l.split(",")]
+            if len(q) < 9:
                 continue
             try:
-                sm.append(float(p[0]))
-                mx = float(p[1])
+                rows.append((t_read, float(q[1]), float(q[2]), q[5:9]))
             except ValueError:
                 continue
-            for n, v in zip(names, p[4:8]):
+        inside = rows
+        in_window = None
+        if self.window and rows:
+            lo, hi = self.window
+            inside = [r for r in rows if lo <= r[0] <= hi + 0.025]
+            in_window = bool(inside)
+            if not inside:                 # window shorter than the period
+                inside = sorted(rows, key=lambda r: min(abs(r[0] - lo), abs(r[0] - hi)))[:2]
+        reasons = set()
+        for r in inside:
+            for n, v in zip(self.NAMES, r[3]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median([r[1] for r in inside]) if inside else None,
+                "sm_max_mhz": inside[-1][2] if inside else None,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "in_timed_window": in_window}
 
 
 def gpu_index(local_rank):
@@ -351,17 +371,20 @@ def main():
             ev_s[j][1].record()
 
     clocks = ClockSampler(gpu_index(local))
+    clocks.start()                       # live before the warm-up ends
     launches0 = 0
+    t_begin = None
     for i in range(Wm + K):
         flush.zero_()
         if i == Wm:
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize()
-            clocks.start()
             launches0 = lib.mla_kernel_launches()
+            t_begin = time.time()
         step(i)
     torch.cuda.synchronize()
+    clocks.mark(t_begin, time.time())
     launches = lib.mla_kernel_launches() - launches0
     if world > 1:
         dist.barrier()

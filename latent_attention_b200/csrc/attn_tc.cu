@@ -15,16 +15,18 @@
 // One CTA = (batch, head, two 128-query tiles A and B); every K/V block it
 // loads serves both tiles.  All query tiles of one head run together
 // (heaviest first), so a head's keys and values leave HBM once.  Warp roles
-// (384 threads):
+// (640 threads):
 //   warp 0       TMA: Q of both tiles (once), K (one stage of 3 boxes)
 //   warp 2       TMA: V ring (2 stages of 2 boxes of 64 value columns)
 //   warp 1       TMEM allocation and MMA issue, in the order
 //                  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
 //                so that the tensor core works on one tile while the other
-//                tile's softmax runs; S_X(j+1) is issued once PV_X(j) has
-//                completed (P_X(j) lives in S_X's columns).
-//   warps 4-7    softmax of tile A, warps 8-11 softmax of tile B (thread =
-//                query row): S from TMEM, causal mask on the diagonal block,
+//                tile's softmax runs; S_X(j+1) follows PV_X(j) in issue order,
+//                which is execution order (P_X(j) lives in S_X's columns).
+//   warps 4-7 / 12-15  softmax of tile A, keys 0-63 / 64-127 of each block;
+//   warps 8-11 / 16-19 the same for tile B (thread = query row and key half;
+//                the halves of a row exchange maxima through shared memory):
+//                S from TMEM, causal mask on the diagonal block,
 //                running max with lazy rescaling (O and l rescaled only when
 //                the max grows by more than 2^8), P as bf16 pairs written
 //                over the first 64 columns of S (the A operand of PV, read
@@ -47,7 +49,7 @@ constexpr int K_BYTES = 3 * BOX;                 // 48 KB per stage
 constexpr int V_BYTES = 2 * BOX;                 // 32 KB
 constexpr int OFF_Q = 0, OFF_K = 2 * Q_BYTES, OFF_V = OFF_K + K_BYTES;
 constexpr int SMEM_BYTES = OFF_V + 2 * V_BYTES + 1024;
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 640;
 constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, DV, 0, 1);   // V is MN-major
 constexpr uint32_t TM_S = 0, TM_O = 256;                   // + 128 * tile
@@ -73,6 +75,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __shared__ __align__(8) uint64_t q_full, k_full, k_empty, v_full[2], v_empty[2], s_full[2],
       p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base;
+  __shared__ float mx_half[2][2][128];   // [tile][key half][row] block maxima
+  __shared__ float l_half[2][2][128];    // [tile][key half][row] final row sums
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[s], 8);          // both key halves' warps
       mbar_init(&pv_done[s], 1);
     }
     mbar_init(&k_full, 1);
@@ -211,9 +215,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (!mbar_wait(&k_full, (j + 1) & 1, abort_v, p.status)) { ok = false; break; }
               k_ready = true;
             }
-            // S_X(j+1) overwrites the columns P_X(j) occupies: wait for PV_X(j)
-            if (!mbar_wait(&pv_done[x], j & 1, abort_v, p.status)) { ok = false; break; }
-            tc_fence_after();
+            // S_X(j+1) overwrites the columns P_X(j) occupies; tcgen05.mma
+            // operations of one thread execute in issue order, so PV_X(j),
+            // issued just before, has read them first
             issue_s(x, j + 1);
           }
         }
@@ -223,8 +227,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp >= 4) {
-    // ---------------- softmax warpgroups: warps 4-7 tile A, 8-11 tile B
-    const int x = warp >= 8 ? 1 : 0;
+    // ---------------- softmax: two warpgroups per tile, one per half of the
+    // 128 keys of a block (warps 4-7 / 12-15 tile A, 8-11 / 16-19 tile B).
+    // The two halves of a row exchange their maxima through shared memory
+    // (named barrier 1 + tile), so both keep the same reference max; each
+    // keeps the row sum of its own keys.
+    const int x = ((warp - 4) >> 2) & 1;             // tile
+    const int hf = (warp - 4) >> 3;                  // key half: columns [64 hf, 64 hf + 64)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;                  // query row within the tile
     const int qi = (x ? q0B : q0A) + r;              // query position
@@ -239,65 +248,66 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // and S_X(j) was issued after PV_X(j-1) completed)
       if (!warp_wait(&s_full[x], j & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, sr[cc]);
+      uint32_t sr[2][32];
+      tmem_ld32(tS + hf * 64, sr[0]);
+      tmem_ld32(tS + hf * 64 + 32, sr[1]);
       tmem_wait_ld();
       // Raw scores; the scale is folded into the exp argument below (scale > 0).
-      const int kmax = min(q_off + qi, Tk - 1) - j * BKV;  // last visible key here
-      if (kmax < 127) {
+      const int kmax = min(q_off + qi, Tk - 1) - j * BKV - hf * 64;  // last visible key here
+      if (kmax < 63) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
+        for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (cc * 32 + i > kmax) sr[cc][i] = __float_as_uint(-INFINITY);
       }
-      float mx8[8];
+      float mx4[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
+      for (int k = 0; k < 4; ++k) mx4[k] = __uint_as_float(sr[0][k]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i)
-        mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[i >> 5][i & 31]));
-      const float mx = fmaxf(m_ref, p.scale_log2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]),
-                                                                fmaxf(mx8[2], mx8[3])),
-                                                          fmaxf(fmaxf(mx8[4], mx8[5]),
-                                                                fmaxf(mx8[6], mx8[7]))));
+      for (int i = 4; i < 64; i += 2)
+        mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], __uint_as_float(sr[i >> 5][i & 31]),
+                                  __uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]));
+      // combine with the other half of the row; after this barrier both halves
+      // have loaded S, so P may be written over it
+      mx_half[x][hf][r] = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+      named_barrier_sync(1 + x, 256);
+      const float mrow = fmaxf(mx_half[x][0][r], mx_half[x][1][r]);
+      const float mx = fmaxf(m_ref, p.scale_log2 * mrow);
       const bool grow = mx > m_ref + kRescaleLog2;    // also true for the first block
       const float alpha = grow ? ex2(m_ref - mx) : 1.f;
       if (grow) {
         l *= alpha;
         m_ref = mx;
       }
-      // P = 2^(scale * s - m_ref) as bf16 pairs over S's first 64 columns
+      // P = 2^(scale * s - m_ref) as bf16 pairs: this half's 64 keys go to
+      // columns [32 hf, 32 hf + 32) of S
       float ls[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
       const float sc = p.scale_log2;
+      uint32_t w[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t w[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int i = half * 64 + 2 * e;
-          const float p0 = ex2(fmaf(__uint_as_float(sr[i >> 5][i & 31]), sc, -m_ref));
-          const float p1 =
-              ex2(fmaf(__uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]), sc, -m_ref));
-          ls[e & 7] += p0 + p1;
-          w[e] = pack_bf16(p0, p1);
-        }
-        tmem_st32(tS + half * 32, w);
+      for (int e = 0; e < 32; ++e) {
+        const int i = 2 * e;
+        const float p0 = ex2(fmaf(__uint_as_float(sr[i >> 5][i & 31]), sc, -m_ref));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]), sc, -m_ref));
+        ls[e & 7] += p0 + p1;
+        w[e] = pack_bf16(p0, p1);
       }
+      tmem_st32(tS + hf * 32, w);
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_X holds the sum through block j-1 (complete, see above)
+        // O_X holds the sum through block j-1 (complete, see above); each half
+        // rescales its 64 of the 128 value columns
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
+          tmem_ld32(tO + hf * 64 + cc * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + cc * 32, o);
+          tmem_st32(tO + hf * 64 + cc * 32, o);
         }
       }
       tmem_wait_st();
@@ -305,15 +315,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[x]);
     }
+    // row sum of both halves; the barrier also keeps the two halves' loops in
+    // step on the exit path
+    l_half[x][hf][r] = l;
+    named_barrier_sync(1 + x, 256);
+    l = l_half[x][0][r] + l_half[x][1][r];
     if (ok && my_nkv > 0 && warp_wait(&pv_done[x], (my_nkv - 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = qi < Tq;
-      __nv_bfloat16* dst = p.o + ((int64_t)(row0 + qi) * p.h + hh) * DV;
+      __nv_bfloat16* dst = p.o + ((int64_t)(row0 + qi) * p.h + hh) * DV + hf * 64;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
+        tmem_ld32(tO + hf * 64 + cc * 32, o);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
