@@ -8,7 +8,9 @@ import ctypes as C
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmla_b200.so")
+# MLA_B200_LIB: another build of the same library (for example a variant to
+# compare against); the default is the in-tree build.
+LIB_PATH = os.environ.get("MLA_B200_LIB") or os.path.join(HERE, "libmla_b200.so")
 
 MLA_OK = 0
 STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_NULL", 2: "MLA_ERR_SHAPE",

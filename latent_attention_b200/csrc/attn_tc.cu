@@ -394,12 +394,10 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
   p.status = a.status;
   p.cu = a.cu_seqlens;
   p.total = a.total;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  static std::atomic<uint64_t> smem_set{0};
+  {
+    const cudaError_t ea = set_dynamic_smem((const void*)attn_tc_kernel, SMEM_BYTES, smem_set);
+    if (ea != cudaSuccess) return ea;
   }
   dim3 grid(p.n_pairs, a.h * a.B);
   attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmKV, tmKpe, p);

@@ -574,12 +574,10 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
     p.part_o = a.part_o;
     p.part_lse = a.part_lse;
     p.status = a.status;
-    static bool attr = false;
-    if (!attr) {
-      e = cudaFuncSetAttribute(latent_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      attr = true;
+    static std::atomic<uint64_t> smem_set{0};
+    {
+      const cudaError_t ea = set_dynamic_smem((const void*)latent_attn_kernel, SMEM_BYTES, smem_set);
+      if (ea != cudaSuccess) return ea;
     }
     dim3 grid(2 * a.B * a.max_splits, 1, (a.h + 127) / 128);
     latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmC, p);

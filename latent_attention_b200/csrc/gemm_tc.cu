@@ -415,12 +415,10 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   p.b_mn = a.b_mn;
   p.sOut = a.sOut;
   p.status = status;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  static std::atomic<uint64_t> smem_set{0};
+  {
+    const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc_kernel, SMEM_BYTES, smem_set);
+    if (ea != cudaSuccess) return ea;
   }
   const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
   gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);

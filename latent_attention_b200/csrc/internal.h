@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <atomic>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -117,6 +118,20 @@ struct DecodeArgs {
   void* o;              // [B, h, dv]
   uint32_t* status;
 };
+
+// cudaFuncSetAttribute applies to the current device only: set a kernel's
+// dynamic shared-memory limit once per device (devices 0..63).
+inline cudaError_t set_dynamic_smem(const void* kernel, int bytes,
+                                    std::atomic<uint64_t>& done_devices) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done_devices.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done_devices.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Launch accounting and stage events (defined in api.cu).
 void count_launches(int n = 1);
