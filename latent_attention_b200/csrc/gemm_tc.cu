@@ -52,6 +52,7 @@ struct TcGemmParams {
   int a_batch_inner, b_mn;
   int64_t sOut;
   int tma_store;          // outputs written by TMA stores (non-batched bf16)
+  int group_m;            // row blocks per raster group
   EpiSeg seg[2];
   uint32_t* status;
 };
@@ -63,8 +64,14 @@ __device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& b
   const int first = p.tiles_m * p.tiles_n[0];
   s = (t >= first) ? 1 : 0;
   const int local = s ? t - first : t;
-  m0 = (local % p.tiles_m) * BM;
-  n0 = (local / p.tiles_m) * BN;
+  // Groups of group_m row blocks: inside a group the row block changes
+  // fastest, so a wave of CTAs shares fewer, fuller A and B panels in L2.
+  const int tn = p.tiles_n[s], G = p.group_m;
+  const int g = local / (G * tn);
+  const int gm = min(G, p.tiles_m - g * G);               // rows of this group
+  const int in = local - g * G * tn;
+  m0 = (g * G + in % gm) * BM;
+  n0 = (in / gm) * BN;
 }
 
 // Epilogue of one 128 x BN tile; this thread owns output row m0 + row.
@@ -411,6 +418,9 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   if (!p.tma_store || a.nseg == 1) tmO[1] = p.tma_store ? tmO[0] : tmA;
   if (!p.tma_store) tmO[0] = tmA;
   p.total_tiles = p.per_batch * a.batch;
+  // long K: grouped raster (measured: o_proj, K = 16384, -0.8 %); short K keeps
+  // the plain column-major order, which the 268 MB kv up-projection prefers
+  p.group_m = a.K >= 4096 ? 16 : p.tiles_m;
   p.a_batch_inner = a.a_batch_inner;
   p.b_mn = a.b_mn;
   p.sOut = a.sOut;
