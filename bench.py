@@ -290,6 +290,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", default=PREFILL,
+                    choices=["dsv3_prefill", "directq_prefill", "kimi_prefill"],
+                    help="prefill workload of the step (default: the headline one)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -316,7 +319,7 @@ def main():
                                 device_id=dev)
     lib = _lib.load()
 
-    wl, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+    wl, wd = WORKLOADS[args.prefill], WORKLOADS[DECODE]
     cfg, cfgd = wl.cfg, wd.cfg
     B, T = wl.batch, wl.seq_len
     seeds = rank_seeds(rank)
@@ -494,7 +497,7 @@ def main():
         dt, done = oracle_prefill_sample(cfg, inp_c, rows)
         cpu = {"value": done / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
                "kind": "oracle",
-               "sample": f"fp64 NumPy oracle on {PREFILL}: keys/values for all {T} "
+               "sample": f"fp64 NumPy oracle on {wl.name}: keys/values for all {T} "
                          f"positions + query/attention/o_proj for 16 rows "
                          f"({done / 1e9:.0f} GFLOP in {dt:.1f} s)"}
 
