@@ -303,7 +303,10 @@ MLA_API mla_status mla_prefill_varlen(const mla_config* cfg, const mla_weights* 
                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes mla_decode_absorbed needs for (cfg, B, max_ctx); 0 if the
- * arguments are invalid.  Fills *layout when it is not NULL. */
+ * arguments are invalid.  Fills *layout when it is not NULL.  The split-KV
+ * length (layout->split_tokens) is 4096 tokens, or shorter (>= 512) when B is
+ * small for the current device's SM count; the result depends on the current
+ * device. */
 MLA_API size_t mla_decode_workspace_size(const mla_config* cfg, int32_t B,
                                  int32_t max_ctx, mla_decode_layout* layout);
 
@@ -333,7 +336,9 @@ MLA_API size_t mla_decode_workspace_size(const mla_config* cfg, int32_t B,
  *   max_ctx       host bound on every ctx_b, >= 1
  *   w_o           NULL, or [hidden, heads*v]
  *   out           [B, heads*v] when w_o is NULL, else [B, hidden]
- *   workspace     >= mla_decode_workspace_size bytes, 256-byte aligned
+ *   workspace     >= mla_decode_workspace_size bytes, 256-byte aligned; a
+ *                 smaller one that fits the layout with 4096-token splits is
+ *                 used with those splits (fewer CTAs for a small batch)
  */
 MLA_API mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope,
                                const void* q_pe, const void* w_kv_b,

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <string>
 
@@ -122,13 +123,37 @@ void prefill_layout(const mla_config& c, int B, int T, int T_past, mla_prefill_l
   L->total_bytes = off;
 }
 
-int decode_split_tokens(const mla_config& c) {
-  return mla::tc_decode_supported(c) ? mla::tc_decode_split_tokens() : 1024;
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  return n;
 }
 
-void decode_layout(const mla_config& c, int B, int max_ctx, mla_decode_layout* L) {
+// Tokens per split of the tensor-core decode.  4096 by default; when the
+// batch yields fewer (sequence, split) pairs than a quarter of the SMs,
+// shorter splits (multiples of 64 tokens, at least 512) give about one CTA
+// pair per pair of SMs.  `fixed` keeps 4096 (the smaller workspace).
+int decode_split_tokens(const mla_config& c, int B, int max_ctx, bool fixed) {
+  if (!mla::tc_decode_supported(c)) return 1024;
+  const int base = mla::tc_decode_split_tokens();
+  if (fixed) return base;
+  const int sms = device_sms();
+  const int64_t items = (int64_t)B * ((max_ctx + base - 1) / base);
+  if (items * 4 >= sms) return base;             // already most of a wave
+  const int64_t want = sms / 2;                  // one CTA pair per SM pair
+  int64_t t = ((int64_t)B * max_ctx + want - 1) / want;
+  t = (t + 63) / 64 * 64;
+  return (int)std::min<int64_t>(base, std::max<int64_t>(512, t));
+}
+
+void decode_layout(const mla_config& c, int B, int max_ctx, mla_decode_layout* L,
+                   bool fixed_split = false) {
   const int64_t es = elem_size(c);
-  const int st = decode_split_tokens(c);
+  const int st = decode_split_tokens(c, B, max_ctx, fixed_split);
   const int ms = (max_ctx + st - 1) / st;
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off = align256(off + bytes); return o; };
@@ -494,11 +519,17 @@ mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope, const 
     return fail(MLA_ERR_ALIGN, "workspace is not 256-byte aligned");
   mla_decode_layout L;
   decode_layout(c, B, max_ctx, &L);
-  if ((int64_t)workspace_bytes < L.total_bytes)
-    return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
-                (long long)L.total_bytes);
-  if (mla::tc_decode_supported(c) && L.max_splits > 64)
-    return fail(MLA_ERR_UNSUPPORTED, "max_ctx=%d needs more than 64 splits", max_ctx);
+  if ((int64_t)workspace_bytes < L.total_bytes) {
+    // a workspace sized for the fixed 4096-token splits still runs
+    mla_decode_layout Lf;
+    decode_layout(c, B, max_ctx, &Lf, true);
+    if ((int64_t)workspace_bytes < Lf.total_bytes)
+      return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
+                  (long long)Lf.total_bytes);
+    L = Lf;
+  }
+  if (mla::tc_decode_supported(c) && L.max_splits > 1024)
+    return fail(MLA_ERR_UNSUPPORTED, "max_ctx=%d needs more than 1024 splits", max_ctx);
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
