@@ -305,62 +305,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
-// Address of the same shared-memory object in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t map_peer(uint32_t local_saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-               ::: "memory");
-}
-
-// Arrive (release, cluster scope) on an mbarrier of another CTA in the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
-               : "memory");
-}
-
-// Relaxed remote arrive: for "buffer consumed" signals whose loads already
-// completed (their values were used before the arrive in program order).
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;"
-      "\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with acquire at cluster scope (for barriers that threads of
-// the peer CTA arrive on after writing into this CTA's shared memory).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint32_t* status) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitNs) {
-        *abort_flag = 1;
-        if (status) atomicOr(status, kStatusTimeout);
-        return false;
-      }
-    }
-  }
-}
-
-
 // Warp-uniform bounded waits: every lane waits, then the lanes agree, so that
 // a timeout seen by one lane never splits the warp before a warp-collective
 // instruction (tcgen05.ld/st, vote).
@@ -368,50 +312,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag, uint32_t* status) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
 }
-__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint32_t* status) {
-  return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity, abort_flag, status));
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                              uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
-               "r"(c), "r"(d)
-               : "memory");
-}
-
-// Asynchronous 16-byte store into another CTA's shared memory that counts its
-// bytes on that CTA's mbarrier (transaction count) when it lands.
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, uint32_t b,
-                                            uint32_t c, uint32_t d, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, "
-      "[%5];" ::"r"(remote_addr),
-      "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
-      : "memory");
-}
-
-// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
-// this CTA's shared memory to a peer CTA's shared memory (a shared::cluster
-// address from map_peer); completion is counted as transaction bytes on the
-// peer's mbarrier `remote_bar`.  No multicast, no global memory.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, uint32_t local_src,
-                                                  uint32_t bytes, uint32_t remote_bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-      "[%3];" ::"r"(remote_dst),
-      "r"(local_src), "r"(bytes), "r"(remote_bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void ld_shared_v4u(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
-                                              uint32_t& d) {
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
-               : "r"(addr)
-               : "memory");
-}
-
 // Prefetch a tensor tile into L2 (no shared memory, no completion signal).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
@@ -452,14 +352,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void ld_shared_v4(uint32_t addr, float& a, float& b, float& c,
-                                             float& d) {
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(a), "=f"(b), "=f"(c), "=f"(d)
-               : "r"(addr)
                : "memory");
 }
 
