@@ -373,3 +373,51 @@ def test_varlen_and_chunked_with_rope_interleave(cuda):
                        generator=g).to(torch.bfloat16)
     out_c, _, _, _ = run_prefill_chunked(cfg, new, past, 150)
     assert oracle.max_rel_err(out_c, oracle.prefill_chunked(cfg, new, past, 150)) <= TOL["bf16"]
+
+
+# --------------------------------------------------------------------------
+# CUDA-graph capture: the C ABI launches only stream work with parameters
+# fixed at the call, so a captured prefill / decode replays bit-identically
+# --------------------------------------------------------------------------
+def _capture(fn):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def test_prefill_and_decode_replay_from_cuda_graphs(cuda):
+    from latent_attention_b200.layer import MlaPrefill, MlaDecode
+    from gpu_helpers import weights_of
+    cfg = small_bf16()
+    inp = make_prefill_inputs(cfg, 2, 300, seed=61)
+    layer = MlaPrefill(cfg, weights_of(inp), 2, 300)
+    x = inp.x.cuda()
+    ref = layer(x).clone()
+    out = torch.empty_like(ref)
+    g = _capture(lambda: layer(x, out=out))
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    layer.check_status()
+
+    dcfg = W["dsv3_decode"].cfg
+    di = make_decode_inputs(dcfg, 4, [1, 700, 4097, 9000], seed=62)
+    dec = MlaDecode(dcfg, 4, 9000)
+    args = [t.cuda() for t in (di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)]
+    dref = torch.empty(4, dcfg.num_heads * dcfg.v_head_dim, dtype=torch.bfloat16, device=cuda)
+    dec(*args, dref)
+    dout = torch.empty_like(dref)
+    gd = _capture(lambda: dec(*args, dout))
+    dout.zero_()
+    gd.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(dout, dref)
+    dec.check_status()
