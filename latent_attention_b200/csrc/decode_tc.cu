@@ -26,9 +26,16 @@
 // every cache byte crosses HBM once.  The same chunk tile is the K-major B
 // operand of S and, for the CTA's 256 latent dims, the MN-major B operand of
 // O += P C.  P_j (bf16 pairs) is written over S_j's TMEM slot.
+// A chunk's boxes form two groups with their own barriers: the 5 boxes only
+// the scores read are released as soon as the first part of S_j has run and
+// are refilled with chunk j+2 while softmax_j and PV_j are still to come; the
+// 4 value boxes of this CTA's latent columns are released by PV_j and read
+// last by S_{j+2}, so their load overlaps the first part of S_{j+2}.
 // Warp roles (384 threads per CTA):
-//   warp 0     TMA: query share once, chunk ring (2 stages), L2 prefetch ahead
+//   warp 0     TMA: query share once, score-only boxes of the chunk ring
+//              (2 stages), L2 prefetch ahead
 //   warp 1     TMEM allocation, MMA issue (S_j or PV, whichever is ready)
+//   warp 2     TMA: the value boxes of the chunk ring
 //   warps 4-7, 8-11  two softmax groups taking alternate chunks (thread =
 //              head), P into TMEM; group 0 also loads the TMEM query part and
 //              writes the epilogue
@@ -64,6 +71,14 @@ constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
 // j % 2), O [128, 384), query dims [0, 256) as bf16 pairs [384, 512).
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_Q = 384;
 constexpr float kRescaleLog2 = 8.f;
+constexpr int SO_BOXES = 5, V_BOXES = 4;      // score-only / value boxes of a chunk
+
+// Box i of the score-only group of the CTA with cluster rank `rank` (the
+// latent half the CTA does not accumulate, then the rope box); the value
+// group of rank c is boxes 4c .. 4c + 3.
+__device__ __forceinline__ int score_only_box(uint32_t rank, int i) {
+  return i < 4 ? (rank ? i : 4 + i) : 8;
+}
 
 struct DecTcParams {
   const int32_t* cu_ctx;
@@ -106,8 +121,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                        const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, qt_full, c_full[NSTAGE], c_empty[NSTAGE],
-      s_full[NSLOT], p_full[NSLOT], pv_done[2], o_done, ref_ready[2], fin;
+  __shared__ __align__(8) uint64_t q_full, qt_full, ca_full[NSTAGE], ca_empty[NSTAGE],
+      cb_full[NSTAGE], cb_empty[NSTAGE], s_full[NSLOT], p_full[NSLOT], pv_done[2], o_done, ref_ready[2], fin;
   __shared__ float m_hand[2][128];          // reference max after chunk j, slot j % 2
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
@@ -136,8 +151,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     mbar_init(&q_full, 1);
     mbar_init(&qt_full, 4);         // softmax group 0 stored the TMEM query part
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&c_full[s], 1);
-      mbar_init(&c_empty[s], 1);
+      mbar_init(&ca_full[s], 1);
+      mbar_init(&ca_empty[s], 1);
+      mbar_init(&cb_full[s], 1);
+      mbar_init(&cb_empty[s], 1);
     }
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(&s_full[s], 1);
@@ -179,12 +196,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (j + PREFETCH < nch)
           for (int a = 0; a < C_ATOMS; ++a)
             tma_prefetch_l2_2d(&tmC, 64 * a, (int)start + chunk_base(n, t0, j + PREFETCH));
-        if (!mbar_wait(&c_empty[st], ((j / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+        if (!mbar_wait(&ca_empty[st], ((j / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
         uint8_t* sc = smem + OFF_C + st * STAGE;
-        mbar_arrive_expect_tx(&c_full[st], C_ATOMS * CBOX);
+        mbar_arrive_expect_tx(&ca_full[st], SO_BOXES * CBOX);
         const int y = (int)start + chunk_base(n, t0, j);
-        for (int a = 0; a < C_ATOMS; ++a)
-          tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &c_full[st]);
+        for (int i = 0; i < SO_BOXES; ++i) {
+          const int a = score_only_box(rank, i);
+          tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &ca_full[st]);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    if (elect_one()) {
+      for (int j = 0; j < nch; ++j) {
+        const int st = j % NSTAGE;
+        if (!mbar_wait(&cb_empty[st], ((j / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+        uint8_t* sc = smem + OFF_C + st * STAGE;
+        mbar_arrive_expect_tx(&cb_full[st], V_BOXES * CBOX);
+        const int y = (int)start + chunk_base(n, t0, j);
+        for (int i = 0; i < V_BOXES; ++i) {
+          const int a = 4 * (int)rank + i;
+          tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &cb_full[st]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -192,33 +225,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_Q));
       bool ok = mbar_wait(&q_full, 0, abort_v, p.status) &&
                 mbar_wait(&qt_full, 0, abort_v, p.status);
+      // S_j += Q box a . C_j box a^T (four MMAs of 16 dims): query dims
+      // [0, 256) from TMEM, the rest from shared memory
+      auto s_box = [&](uint32_t d, uint64_t dc, int a, bool first) {
+        if (a < QT_ATOMS) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ts(d, tbase + TM_Q + a * 32 + k * 8,
+                        dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(d, dq + (uint64_t)(((a - QT_ATOMS) * QBOX + k * 32) >> 4),
+                     dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
+        }
+      };
       // Issue S_js and O += P_jp C_jp in whichever order their inputs become
       // ready.  S_js reuses the slot of S/P_{js-2}, so it follows PV_{js-2} in
       // issue order (js < jp + 2), which is execution order; PV_jp follows S_jp.
+      // S_js goes out in two parts: the score-only boxes, then the value boxes.
       int js = 0, jp = 0;
+      bool s_part = false;                 // S_js's score-only part is issued
       const uint64_t t_start = globaltimer();
       uint32_t idle = 0;
       while (ok && jp < nch) {
         bool progress = false;
         if (js < nch && js < jp + NSLOT) {
           const int st = js % NSTAGE, sl = js % NSLOT;
-          if (mbar_test(&c_full[st], (js / NSTAGE) & 1)) {
+          const uint32_t par = (js / NSTAGE) & 1;
+          const uint32_t d = tbase + TM_S + sl * NT;
+          const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
+          if (!s_part && mbar_test(&ca_full[st], par)) {
             tc_fence_after();
-            const uint32_t d = tbase + TM_S + sl * NT;
-            const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
-#pragma unroll
-            for (int a = 0; a < QT_ATOMS; ++a)      // dims [0, 256): A from TMEM
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts(d, tbase + TM_Q + a * 32 + k * 8,
-                            dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, (a | k) != 0);
-#pragma unroll
-            for (int a = 0; a < QS_ATOMS; ++a)      // dims [256, 576): A from shared memory
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16(d, dq + (uint64_t)((a * QBOX + k * 32) >> 4),
-                         dc + (uint64_t)(((QT_ATOMS + a) * CBOX + k * 32) >> 4), IDESC_S, 1);
+            for (int i = 0; i < SO_BOXES; ++i) s_box(d, dc, score_only_box(rank, i), i == 0);
+            mma_commit(&ca_empty[st]);
+            s_part = true;
+            progress = true;
+          }
+          if (s_part && mbar_test(&cb_full[st], par)) {
+            tc_fence_after();
+            for (int i = 0; i < V_BOXES; ++i) s_box(d, dc, 4 * (int)rank + i, false);
             mma_commit(&s_full[sl]);
+            s_part = false;
             ++js;
             progress = true;
           }
@@ -233,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             for (int k = 0; k < NT / 16; ++k)
               mma_bf16_ts(tbase + TM_O, tbase + TM_S + sl * NT + k * 8,
                           dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (jp | k) != 0);
-            mma_commit(&c_empty[st]);
+            mma_commit(&cb_empty[st]);
             mma_commit(&pv_done[jp & 1]);
             if (jp == nch - 1) mma_commit(&o_done);
             ++jp;
