@@ -150,7 +150,9 @@ typedef struct mla_prefill_layout {
 /* Byte offsets of the decode intermediates inside the workspace:
  *   q_lat  [B, heads, kv_lora+rope] absorbed query (W_UK^T q_nope | q_pe)
  *   o_lat  [B, heads, kv_lora]      attention output in latent space
- *   part_o / part_lse               split-KV partial results
+ *   part_o / part_lse               partial results of split sequences
+ *                                   ([max_splits, heads, ...] on tensor
+ *                                   cores, [B, max_splits, heads, ...] else)
  *   o      [B, heads, v]            output before the optional o_proj */
 typedef struct mla_decode_layout {
   int64_t status, q_lat, part_o, part_lse, o_lat, o, total_bytes;
@@ -303,10 +305,14 @@ MLA_API mla_status mla_prefill_varlen(const mla_config* cfg, const mla_weights* 
                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes mla_decode_absorbed needs for (cfg, B, max_ctx); 0 if the
- * arguments are invalid.  Fills *layout when it is not NULL.  The split-KV
- * length (layout->split_tokens) is 4096 tokens, or shorter (>= 512) when B is
- * small for the current device's SM count; the result depends on the current
- * device. */
+ * arguments are invalid.  Fills *layout when it is not NULL.
+ * Tensor-core configurations (bf16, kv_lora_rank 512, rope 64): the tokens of
+ * all sequences, concatenated, are cut into equal slices of at least
+ * layout->split_tokens tokens, one per pair of SMs; a sequence that crosses
+ * a slice boundary leaves one partial result per slice, in one of
+ * layout->max_splits slots (two per SM pair).  The result depends on the
+ * current device's SM count.  Other configurations: split_tokens-token
+ * splits of every sequence, max_splits of them per sequence. */
 MLA_API size_t mla_decode_workspace_size(const mla_config* cfg, int32_t B,
                                  int32_t max_ctx, mla_decode_layout* layout);
 
@@ -336,9 +342,9 @@ MLA_API size_t mla_decode_workspace_size(const mla_config* cfg, int32_t B,
  *   max_ctx       host bound on every ctx_b, >= 1
  *   w_o           NULL, or [hidden, heads*v]
  *   out           [B, heads*v] when w_o is NULL, else [B, hidden]
- *   workspace     >= mla_decode_workspace_size bytes, 256-byte aligned; a
- *                 smaller one that fits the layout with 4096-token splits is
- *                 used with those splits (fewer CTAs for a small batch)
+ *   workspace     mla_decode_workspace_size bytes, 256-byte aligned; on
+ *                 tensor cores a smaller one runs on as many SM pairs as its
+ *                 partial slots allow (MLA_ERR_WORKSPACE below one pair)
  */
 MLA_API mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope,
                                const void* q_pe, const void* w_kv_b,
@@ -401,9 +407,10 @@ MLA_API int64_t mla_kernel_launches(void);
  *
  *   Arguments, layouts and results are those of mla_decode_absorbed without
  *   the workspace pair.
- *   Returns MLA_ERR_WORKSPACE (with mla_last_error_detail naming both sizes)
- *   when mla_decode_workspace_size(cfg, B, max_ctx) exceeds the array, e.g.
- *   B = 16 sequences of 128 heads up to max_ctx = 8192 fit; B = 64 does not.
+ *   The array holds the partial slots of fewer SM pairs than a full
+ *   workspace, so the decode may run on fewer SMs.  Returns MLA_ERR_WORKSPACE
+ *   (with mla_last_error_detail naming both sizes) when not even one pair's
+ *   layout fits, e.g. B = 16 sequences of 128 heads fit; B = 64 do not.
  *   The first call on each device looks up that device's copy of the array
  *   (cudaGetSymbolAddress) and caches it; make that first call before any
  *   stream capture.  The call allocates nothing: no cudaMalloc, cudaFree or

@@ -133,40 +133,48 @@ int device_sms() {
   return n;
 }
 
-// Tokens per split of the tensor-core decode.  4096 by default; when the
-// batch yields fewer (sequence, split) pairs than a quarter of the SMs,
-// shorter splits (multiples of 64 tokens, at least 512) give about one CTA
-// pair per pair of SMs.  `fixed` keeps 4096 (the smaller workspace).
-int decode_split_tokens(const mla_config& c, int B, int max_ctx, bool fixed) {
-  if (!mla::tc_decode_supported(c)) return 1024;
-  const int base = mla::tc_decode_split_tokens();
-  if (fixed) return base;
-  const int sms = device_sms();
-  const int64_t items = (int64_t)B * ((max_ctx + base - 1) / base);
-  if (items * 4 >= sms) return base;             // already most of a wave
-  const int64_t want = sms / 2;                  // one CTA pair per SM pair
-  int64_t t = ((int64_t)B * max_ctx + want - 1) / want;
-  t = (t + 63) / 64 * 64;
-  return (int)std::min<int64_t>(base, std::max<int64_t>(512, t));
-}
-
-void decode_layout(const mla_config& c, int B, int max_ctx, mla_decode_layout* L,
-                   bool fixed_split = false) {
+// Decode partitions.  Tensor cores: one CTA pair per two SMs, each taking an
+// equal slice (at least tc_decode_min_slice() tokens) of all sequences'
+// tokens; a sequence that crosses a slice boundary leaves one partial per
+// slice in one of 2 slots per pair (split_tokens = the shortest slice,
+// max_splits = the slot count).  SIMT: 1024-token splits of every sequence
+// (max_splits per sequence).
+// `units` > 0 asks for that many SM pairs (tensor cores) instead of one per
+// two SMs of the current device.
+void decode_layout(const mla_config& c, int B, int max_ctx, mla_decode_layout* L, int units = 0) {
   const int64_t es = elem_size(c);
-  const int st = decode_split_tokens(c, B, max_ctx, fixed_split);
-  const int ms = (max_ctx + st - 1) / st;
+  int64_t parts;
+  if (mla::tc_decode_supported(c)) {
+    L->split_tokens = mla::tc_decode_min_slice();
+    L->max_splits = 2 * (units > 0 ? units : std::max(1, device_sms() / 2));
+    parts = L->max_splits;
+  } else {
+    L->split_tokens = 1024;
+    L->max_splits = (max_ctx + 1023) / 1024;
+    parts = (int64_t)B * L->max_splits;
+  }
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off = align256(off + bytes); return o; };
-  L->split_tokens = st;
-  L->max_splits = ms;
   L->status = take(256);
   L->q_lat = take((int64_t)B * c.num_heads * (c.kv_lora_rank + c.qk_rope_head_dim) * es);
-  L->part_o = take((int64_t)B * ms * c.num_heads * c.kv_lora_rank * 4);
-  L->part_lse = take((int64_t)B * ms * c.num_heads * 4);
+  L->part_o = take(parts * c.num_heads * c.kv_lora_rank * 4);
+  L->part_lse = take(parts * c.num_heads * 4);
   L->o_lat = take((int64_t)B * c.num_heads * c.kv_lora_rank * es);
   L->o = take((int64_t)B * c.num_heads * c.v_head_dim * es);
   L->total_bytes = off;
 }
+
+}  // namespace
+
+namespace mla {
+size_t decode_min_workspace(const mla_config& c, int B, int max_ctx) {
+  mla_decode_layout L;
+  decode_layout(c, B, max_ctx, &L, mla::tc_decode_supported(c) ? 1 : 0);
+  return (size_t)L.total_bytes;
+}
+}  // namespace mla
+
+namespace {
 
 char* at(void* ws, int64_t off) { return off < 0 ? nullptr : static_cast<char*>(ws) + off; }
 
@@ -519,17 +527,16 @@ mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope, const 
     return fail(MLA_ERR_ALIGN, "workspace is not 256-byte aligned");
   mla_decode_layout L;
   decode_layout(c, B, max_ctx, &L);
-  if ((int64_t)workspace_bytes < L.total_bytes) {
-    // a workspace sized for the fixed 4096-token splits still runs
-    mla_decode_layout Lf;
-    decode_layout(c, B, max_ctx, &Lf, true);
-    if ((int64_t)workspace_bytes < Lf.total_bytes)
-      return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
-                  (long long)Lf.total_bytes);
-    L = Lf;
+  if ((int64_t)workspace_bytes < L.total_bytes && mla::tc_decode_supported(c)) {
+    // a smaller workspace runs on as many SM pairs as its partial slots allow
+    for (int u = L.max_splits / 2 - 1; u >= 1; --u) {
+      decode_layout(c, B, max_ctx, &L, u);
+      if ((int64_t)workspace_bytes >= L.total_bytes) break;
+    }
   }
-  if (mla::tc_decode_supported(c) && L.max_splits > 1024)
-    return fail(MLA_ERR_UNSUPPORTED, "max_ctx=%d needs more than 1024 splits", max_ctx);
+  if ((int64_t)workspace_bytes < L.total_bytes)
+    return fail(MLA_ERR_WORKSPACE, "workspace %zu < %lld bytes", workspace_bytes,
+                (long long)L.total_bytes);
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
@@ -541,6 +548,7 @@ mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope, const 
   a.dr = c.qk_rope_head_dim; a.dv = c.v_head_dim; a.r = c.kv_lora_rank;
   a.scale = (float)softmax_scale(c);
   a.split_tokens = L.split_tokens; a.max_splits = L.max_splits;
+  a.n_units = L.max_splits / 2; a.min_len = L.split_tokens;
   a.q_lat = at(ws, L.q_lat); a.part_o = (float*)at(ws, L.part_o);
   a.part_lse = (float*)at(ws, L.part_lse); a.o_lat = at(ws, L.o_lat);
   a.o = w_o ? at(ws, L.o) : out;

@@ -30,8 +30,10 @@ mla_status mla_decode_absorbed_noalloc(const mla_config* cfg, const void* q_nope
                                        const int32_t* cu_ctx, int32_t B, int32_t max_ctx,
                                        const void* w_o, void* out, void* stream) {
   if (!cfg) return MLA_ERR_NULL;
-  const size_t need = mla_decode_workspace_size(cfg, B, max_ctx, nullptr);
-  if (need == 0) return MLA_ERR_SHAPE;
+  if (mla_decode_workspace_size(cfg, B, max_ctx, nullptr) == 0) return MLA_ERR_SHAPE;
+  // the array may hold fewer partial slots than the full layout: the decode
+  // then runs on fewer SM pairs
+  const size_t need = mla::decode_min_workspace(*cfg, B, max_ctx);
   if (need > (size_t)MLA_DECODE_NOALLOC_SCRATCH_BYTES) {
     char msg[160];
     snprintf(msg, sizeof(msg), "decode needs %zu scratch bytes; the static array holds %zu",

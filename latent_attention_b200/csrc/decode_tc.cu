@@ -8,37 +8,51 @@
 //   D1 q_lat[b,h] = W_UK[h]^T q_nope[b,h]          batched tcgen05 GEMM (one
 //                                                   product per head, W_UK read
 //                                                   as an MN-major operand)
-//   D2 latent_attn_kernel  split-KV attention of the 128 heads of a sequence
-//                          over its [ctx, 576] cache, on tcgen05 (below)
-//   D3 combine_kernel      log-sum-exp merge of the splits -> o_lat (bf16)
+//   D2 latent_attn_kernel  attention of the 128 heads of a sequence over its
+//                          [ctx, 576] cache, on tcgen05 (below)
+//   D3 combine_kernel      log-sum-exp merge of the partial results of the
+//                          sequences D2 split -> o_lat (bf16)
 //   D4 o[b,h] = W_UV[h] o_lat[b,h]                  batched tcgen05 GEMM
 //
+// D2 schedule.  The tokens of all sequences, concatenated in cu_ctx order,
+// are cut into equal slices, one per CTA pair ("unit", one pair per two
+// SMs, a single wave), so every unit has the same number of cache rows to
+// read whatever the length mix.  A unit walks the segments of its slice (the
+// parts of the sequences inside it) with one continuous chunk pipeline; a
+// segment covering a whole sequence writes o_lat itself, the first and last
+// segment of a slice leave a partial (o, lse) for D3.
+//
 // D2 design.  With 128 heads as the MMA M dimension the latent output
-// O[128, 512] in fp32 fills all 512 TMEM columns, so a cluster of two CTAs
-// shares one (sequence, split): CTA c accumulates latent columns
-// [256c, 256c+256) of O (256 TMEM columns).  Each CTA computes the full
-// scores S = Q C^T over all 576 cached dims itself -- the query's latent
-// dims [0, 256) sit in TMEM (A operand from tensor memory, 128 columns), the
-// rest (latent [256, 512) and rope) in shared memory -- so the two CTAs need
-// no partial-score exchange and run the identical online softmax.  Each CTA
-// TMA-loads every 64-token chunk in full (9 boxes of 64 dims): the pair reads
-// the same rows at the same time, so the second read is served by L2 and
-// every cache byte crosses HBM once.  The same chunk tile is the K-major B
-// operand of S and, for the CTA's 256 latent dims, the MN-major B operand of
-// O += P C.  P_j (bf16 pairs) is written over S_j's TMEM slot.
+// O[128, 512] in fp32 fills all 512 TMEM columns, so the two CTAs of a unit
+// split it: CTA c accumulates latent columns [256c, 256c+256) of O (256 TMEM
+// columns).  Each CTA computes the full scores S = Q C^T over all 576 cached
+// dims itself -- the query's latent dims [0, 256) sit in TMEM (A operand from
+// tensor memory, 128 columns), the rest (latent [256, 512) and rope) in
+// shared memory -- so the two CTAs need no partial-score exchange and run the
+// identical online softmax.  Each CTA TMA-loads every 64-token chunk in full
+// (9 boxes of 64 dims): the pair reads the same rows at the same time, so the
+// second read is served by L2 and every cache byte crosses HBM once.  The
+// same chunk tile is the K-major B operand of S and, for the CTA's 256 latent
+// dims, the MN-major B operand of O += P C.  P_g (bf16 pairs) is written over
+// S_g's TMEM slot.
 // A chunk's boxes form two groups with their own barriers: the 5 boxes only
-// the scores read are released as soon as the first part of S_j has run and
-// are refilled with chunk j+2 while softmax_j and PV_j are still to come; the
-// 4 value boxes of this CTA's latent columns are released by PV_j and read
-// last by S_{j+2}, so their load overlaps the first part of S_{j+2}.
+// the scores read are released as soon as the first part of S_g has run and
+// are refilled with chunk g+2 while softmax_g and PV_g are still to come; the
+// 4 value boxes of this CTA's latent columns are released by PV_g and read
+// last by S_{g+2}, so their load overlaps the first part of S_{g+2}.
+// Between segments the query changes: the next segment's first S waits for
+// its query (the shared-memory part is reloaded once the previous segment's
+// epilogue, which stages its TMA stores in the query buffer, is done; the
+// TMEM part once the previous segment's last S has completed), and its first
+// PV for the previous O to have been read out.
 // Warp roles (384 threads per CTA):
-//   warp 0     TMA: query share once, score-only boxes of the chunk ring
-//              (2 stages), L2 prefetch ahead
-//   warp 1     TMEM allocation, MMA issue (S_j or PV, whichever is ready)
+//   warp 0     TMA: each segment's query share, score-only boxes of the chunk
+//              ring (2 stages), L2 prefetch ahead (into the next segment)
+//   warp 1     TMEM allocation, MMA issue (S_g or PV, whichever is ready)
 //   warp 2     TMA: the value boxes of the chunk ring
 //   warps 4-7, 8-11  two softmax groups taking alternate chunks (thread =
-//              head), P into TMEM; group 0 also loads the TMEM query part and
-//              writes the epilogue
+//              head), P into TMEM; group 1 also stores each segment's TMEM
+//              query part, group 0 writes each segment's result
 // All waits are bounded; a timeout sets the device status word.
 #include <cfloat>
 
@@ -72,6 +86,7 @@ constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_Q = 384;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int SO_BOXES = 5, V_BOXES = 4;      // score-only / value boxes of a chunk
+constexpr int EPI_BOX = 32 * 128;             // epilogue staging: 32 rows of 128 bytes
 
 // Box i of the score-only group of the CTA with cluster rank `rank` (the
 // latent half the CTA does not accumulate, then the rope box); the value
@@ -84,24 +99,13 @@ struct DecTcParams {
   const int32_t* cu_ctx;
   const __nv_bfloat16* q_lat;  // [B, h, 512]
   int B, h, max_ctx;
-  int split_tokens, max_splits;
+  int n_units, min_len;        // CTA pairs; shortest slice of the token stream
   float scale_log2;
-  float* part_o;      // [B, max_splits, h, R]
-  float* part_lse;    // [B, max_splits, h]
+  float* part_o;               // [2 n_units, h, R]
+  float* part_lse;             // [2 n_units, h]
+  __nv_bfloat16* o_lat;        // [B, h, R]
   uint32_t* status;
 };
-
-__device__ __forceinline__ int seq_len(const int32_t* cu, int b, int max_ctx, uint32_t* status,
-                                       int64_t* start) {
-  const int64_t s = cu[b], e = cu[b + 1];
-  int64_t n = e - s;
-  if (n < 1 || n > max_ctx) {
-    if (threadIdx.x == 0) atomicOr(status, kStatusBadCtx);
-    n = n < 1 ? 0 : max_ctx;
-  }
-  *start = s;
-  return (int)n;
-}
 
 // First token (relative to the sequence start) of the 64-row box that chunk j
 // of a split starting at token t0 loads.  A box never reaches past the last
@@ -115,41 +119,133 @@ __device__ __forceinline__ int chunk_base(int n, int t0, int j) {
   return n >= NT ? min(lt, n - NT) : n - NT;
 }
 
+// The token stream of all sequences, concatenated in cu_ctx order, is cut
+// into equal slices of L tokens, one per CTA pair ("unit"); L is at least
+// min_len.  A unit's segment of sequence b is the part of b inside its
+// slice.  A segment that covers all of b is written to o_lat directly; any
+// other segment leaves a partial (o, lse) in slot 2u (the unit's first
+// segment) or 2u + 1 (its last), which the combine kernel merges.
+struct Slice {
+  int64_t r0, r1, L;   // tokens [r0, r1) of the stream, relative to cu_ctx[0]
+};
+
+__device__ __forceinline__ Slice unit_slice(const int32_t* cu, int B, int max_ctx, int u,
+                                            int n_units, int min_len) {
+  const int64_t T = min(max((int64_t)cu[B] - cu[0], (int64_t)0), (int64_t)B * max_ctx);
+  const int64_t L = max((T + n_units - 1) / n_units, (int64_t)min_len);
+  Slice s;
+  s.L = L;
+  s.r0 = min((int64_t)u * L, T);
+  s.r1 = min(s.r0 + L, T);
+  return s;
+}
+
+// First sequence whose tokens reach past stream position r (cu_ctx is
+// non-decreasing for valid input; any input gives an index in [0, B)).
+__device__ __forceinline__ int seq_at(const int32_t* cu, int B, int64_t r) {
+  int lo = 0, hi = B - 1;
+  const int64_t c0 = cu[0];
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)cu[mid + 1] - c0 <= r) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+struct Seg {
+  int b, n, t0, tcount, nch, slot;
+  int64_t start;       // cache row of the sequence's token 0
+  bool whole;          // the segment covers the whole sequence
+};
+
+// Segment of sequence b in the slice of unit u; nch = 0 when it is empty or
+// the sequence is invalid (the combine kernel reports those).
+__device__ __forceinline__ Seg seg_info(const int32_t* cu, int b, int max_ctx, const Slice& sl,
+                                        int u) {
+  Seg s;
+  s.b = b;
+  const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
+  s.start = cu[b];
+  const int64_t n = ce - cb;
+  const int64_t s0 = max(sl.r0, cb), s1 = min(sl.r1, ce);
+  s.n = (int)min(max(n, (int64_t)0), (int64_t)max_ctx);
+  s.t0 = (int)max(s0 - cb, (int64_t)0);
+  s.tcount = (int)max(s1 - s0, (int64_t)0);
+  if (n < 1 || n > max_ctx) s.tcount = 0;
+  s.nch = (s.tcount + NT - 1) / NT;
+  s.whole = s.t0 == 0 && s.tcount == n;
+  s.slot = 2 * u + (cb > sl.r0 ? 1 : 0);
+  return s;
+}
+
+// Walks the non-empty segments of a unit in order.
+struct SegCursor {
+  int k, kk;           // sequence offset from b0, ordinal among non-empty segments
+  int j;               // chunk within the segment
+  Seg s;
+  bool done;
+  __device__ __forceinline__ void seek(const int32_t* cu, int b0, int b1, int max_ctx,
+                                       const Slice& sl, int u) {
+    for (; b0 + k < b1; ++k) {
+      s = seg_info(cu, b0 + k, max_ctx, sl, u);
+      if (s.nch > 0) { done = false; return; }
+    }
+    done = true;
+  }
+  __device__ __forceinline__ void start(const int32_t* cu, int b0, int b1, int max_ctx,
+                                        const Slice& sl, int u) {
+    k = 0; kk = 0; j = 0;
+    seek(cu, b0, b1, max_ctx, sl, u);
+  }
+  __device__ __forceinline__ void next_seg(const int32_t* cu, int b0, int b1, int max_ctx,
+                                           const Slice& sl, int u) {
+    j = 0; ++k; ++kk;
+    seek(cu, b0, b1, max_ctx, sl, u);
+  }
+  // next chunk; true when it starts a new segment
+  __device__ __forceinline__ bool next(const int32_t* cu, int b0, int b1, int max_ctx,
+                                       const Slice& sl, int u) {
+    if (++j < s.nch) return false;
+    j = 0; ++k; ++kk;
+    seek(cu, b0, b1, max_ctx, sl, u);
+    return true;
+  }
+};
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmQpe,
                        const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmPO,
+                       const __grid_constant__ CUtensorMap tmOL,
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, qt_full, ca_full[NSTAGE], ca_empty[NSTAGE],
-      cb_full[NSTAGE], cb_empty[NSTAGE], s_full[NSLOT], p_full[NSLOT], pv_done[2], o_done, ref_ready[2], fin;
-  __shared__ float m_hand[2][128];          // reference max after chunk j, slot j % 2
+  __shared__ __align__(8) uint64_t q_full, qt_full, q_free, ca_full[NSTAGE], ca_empty[NSTAGE],
+      cb_full[NSTAGE], cb_empty[NSTAGE], s_full[NSLOT], p_full[NSLOT], pv_done[2], o_done,
+      o_free, ref_ready[2];
+  __shared__ float m_hand[128];                // reference max after the last chunk
+  __shared__ float fin_m[128], fin_l[128];      // group 1's state at a segment's end
   __shared__ uint32_t tmem_base;
-  __shared__ int abort_flag;
+  __shared__ int abort_flag, seq_lo, seq_hi;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_v = &abort_flag;
 
   const uint32_t rank = cluster_rank();
-  const int item = blockIdx.x >> 1;
-  const int b = item / p.max_splits, sp = item % p.max_splits;
+  const int u = blockIdx.x >> 1;
   const int h0 = blockIdx.z * 128;
-  int64_t start;
-  const int n = seq_len(p.cu_ctx, b, p.max_ctx, p.status, &start);
-  const int t0 = sp * p.split_tokens;
-  if (t0 >= n) {   // empty split (both CTAs of the pair take this branch)
-    if (rank == 0 && threadIdx.x < 128 && h0 + threadIdx.x < p.h)
-      p.part_lse[((int64_t)b * p.max_splits + sp) * p.h + h0 + threadIdx.x] = -INFINITY;
-    return;
-  }
-  const int tcount = min(p.split_tokens, n - t0);
-  const int nch = (tcount + NT - 1) / NT;
+  const int32_t* cu = p.cu_ctx;
+  const Slice sl = unit_slice(cu, p.B, p.max_ctx, u, p.n_units, p.min_len);
+  if (sl.r0 >= sl.r1) return;                    // past the end of the stream (both CTAs)
   const int dim0 = 256 * (int)rank;              // this CTA's latent columns of O
 
   if (threadIdx.x == 0) {
+    seq_lo = seq_at(cu, p.B, sl.r0);
+    seq_hi = seq_at(cu, p.B, sl.r1 - 1) + 1;
     mbar_init(&q_full, 1);
-    mbar_init(&qt_full, 4);         // softmax group 0 stored the TMEM query part
+    mbar_init(&qt_full, 4);         // softmax group 1 stored the TMEM query part
+    mbar_init(&q_free, 1);          // the last S of a segment completed
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&ca_full[s], 1);
       mbar_init(&ca_empty[s], 1);
@@ -158,14 +254,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);     // the chunk's softmax group wrote P_j
+      mbar_init(&p_full[s], 4);     // the chunk's softmax group wrote P_g
     }
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
-    mbar_init(&o_done, 1);
-    mbar_init(&ref_ready[0], 4);    // a softmax group published chunk j's reference
+    mbar_init(&o_done, 1);          // the last PV of a segment completed
+    mbar_init(&o_free, 4);          // softmax group 0 has read O out of TMEM
+    mbar_init(&ref_ready[0], 4);    // a softmax group published chunk g's reference
     mbar_init(&ref_ready[1], 4);
-    mbar_init(&fin, 4);             // softmax group 1 published its final sum
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -176,57 +272,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tmem_base;
+  const int b0 = seq_lo, b1 = seq_hi;
   // softmax groups: warps 4..7 (group 0) and 8..11 (group 1)
   const int sm_wg = (warp >= 4 && warp < 8) ? 0 : (warp >= 8 ? 1 : -1);
 
   if (warp == 0) {
+    // ---------------- query share of each segment, score-only boxes, L2 prefetch
     if (elect_one()) {
       tma_prefetch(&tmQ);
       tma_prefetch(&tmQpe);
       tma_prefetch(&tmC);
-      mbar_arrive_expect_tx(&q_full, QS_ATOMS * QBOX);
-      for (int a = 0; a < 4; ++a)      // query latent dims [256, 512)
-        tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, 256 + 64 * a, b * p.h + h0, &q_full);
-      tma_load_2d(smem + OFF_Q + 4 * QBOX, &tmQpe, 0, b * p.h + h0, &q_full);
-      for (int j = 0; j < PREFETCH && j < nch; ++j)
+      auto prefetch = [&](const Seg& s, int j) {
         for (int a = 0; a < C_ATOMS; ++a)
-          tma_prefetch_l2_2d(&tmC, 64 * a, (int)start + chunk_base(n, t0, j));
-      for (int j = 0; j < nch; ++j) {
-        const int st = j % NSTAGE;
-        if (j + PREFETCH < nch)
-          for (int a = 0; a < C_ATOMS; ++a)
-            tma_prefetch_l2_2d(&tmC, 64 * a, (int)start + chunk_base(n, t0, j + PREFETCH));
-        if (!mbar_wait(&ca_empty[st], ((j / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+          tma_prefetch_l2_2d(&tmC, 64 * a, (int)s.start + chunk_base(s.n, s.t0, j));
+      };
+      // the query rows of a segment (all 576 dims) into L2
+      auto prefetch_q = [&](const Seg& s) {
+        for (int a = 0; a < 8; ++a) tma_prefetch_l2_2d(&tmQ, 64 * a, s.b * p.h + h0);
+        tma_prefetch_l2_2d(&tmQpe, 0, s.b * p.h + h0);
+      };
+      SegCursor c, nx;
+      c.start(cu, b0, b1, p.max_ctx, sl, u);
+      int prev_nch = 0;
+      for (int g = 0; !c.done; ++g) {
+        const Seg& s = c.s;
+        if (c.j == 0) {
+          if (prev_nch < PREFETCH)         // not prefetched by the previous segment
+            for (int j = 0; j < PREFETCH && j < s.nch; ++j) prefetch(s, j);
+          prev_nch = s.nch;
+          nx = c;                          // the next segment, prefetched near this one's end
+          nx.next_seg(cu, b0, b1, p.max_ctx, sl, u);
+          // the previous segment's epilogue has finished with the query buffer
+          if (c.kk > 0 && !mbar_wait(&o_free, (c.kk - 1) & 1, abort_v, p.status)) break;
+          mbar_arrive_expect_tx(&q_full, QS_ATOMS * QBOX);
+          for (int a = 0; a < 4; ++a)      // query latent dims [256, 512)
+            tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, 256 + 64 * a, s.b * p.h + h0, &q_full);
+          tma_load_2d(smem + OFF_Q + 4 * QBOX, &tmQpe, 0, s.b * p.h + h0, &q_full);
+        }
+        if (c.j + PREFETCH < s.nch) {
+          prefetch(s, c.j + PREFETCH);
+        } else if (!nx.done) {
+          const int jn = c.j + PREFETCH - s.nch;
+          if (jn == 0) prefetch_q(nx.s);
+          if (jn < nx.s.nch) prefetch(nx.s, jn);
+        }
+        const int st = g % NSTAGE;
+        if (!mbar_wait(&ca_empty[st], ((g / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
         uint8_t* sc = smem + OFF_C + st * STAGE;
         mbar_arrive_expect_tx(&ca_full[st], SO_BOXES * CBOX);
-        const int y = (int)start + chunk_base(n, t0, j);
+        const int y = (int)s.start + chunk_base(s.n, s.t0, c.j);
         for (int i = 0; i < SO_BOXES; ++i) {
           const int a = score_only_box(rank, i);
           tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &ca_full[st]);
         }
+        c.next(cu, b0, b1, p.max_ctx, sl, u);
       }
     }
   } else if (warp == 2) {
+    // ---------------- value boxes
     if (elect_one()) {
-      for (int j = 0; j < nch; ++j) {
-        const int st = j % NSTAGE;
-        if (!mbar_wait(&cb_empty[st], ((j / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+      SegCursor c;
+      c.start(cu, b0, b1, p.max_ctx, sl, u);
+      for (int g = 0; !c.done; ++g) {
+        const Seg& s = c.s;
+        const int st = g % NSTAGE;
+        if (!mbar_wait(&cb_empty[st], ((g / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
         uint8_t* sc = smem + OFF_C + st * STAGE;
         mbar_arrive_expect_tx(&cb_full[st], V_BOXES * CBOX);
-        const int y = (int)start + chunk_base(n, t0, j);
+        const int y = (int)s.start + chunk_base(s.n, s.t0, c.j);
         for (int i = 0; i < V_BOXES; ++i) {
           const int a = 4 * (int)rank + i;
           tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &cb_full[st]);
         }
+        c.next(cu, b0, b1, p.max_ctx, sl, u);
       }
     }
   } else if (warp == 1) {
+    // ---------------- MMA issue
     if (elect_one()) {
       const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_Q));
-      bool ok = mbar_wait(&q_full, 0, abort_v, p.status) &&
-                mbar_wait(&qt_full, 0, abort_v, p.status);
-      // S_j += Q box a . C_j box a^T (four MMAs of 16 dims): query dims
-      // [0, 256) from TMEM, the rest from shared memory
+      // S_g += Q box a . C_g box a^T (four MMAs of 16 dims): query dims
+      // [0, 256) from TMEM, the rest from shared memory; dc describes the
+      // chunk's stage
       auto s_box = [&](uint32_t d, uint64_t dc, int a, bool first) {
         if (a < QT_ATOMS) {
 #pragma unroll
@@ -240,22 +367,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                      dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
         }
       };
-      // Issue S_js and O += P_jp C_jp in whichever order their inputs become
-      // ready.  S_js reuses the slot of S/P_{js-2}, so it follows PV_{js-2} in
-      // issue order (js < jp + 2), which is execution order; PV_jp follows S_jp.
-      // S_js goes out in two parts: the score-only boxes, then the value boxes.
-      int js = 0, jp = 0;
-      bool s_part = false;                 // S_js's score-only part is issued
-      const uint64_t t_start = globaltimer();
+      // Issue S_gs and O += P_gp C_gp in whichever order their inputs become
+      // ready, across segments.  S_gs reuses the slot of S/P_{gs-2}, so it
+      // follows PV_{gs-2} in issue order (gs < gp + 2), which is execution
+      // order; PV_gp follows S_gp.  S_gs goes out in two parts: the
+      // score-only boxes, then the value boxes.  A segment's first S waits
+      // for its query (shared memory and TMEM parts), its first PV for the
+      // previous segment's O to have been read out.
+      SegCursor cs, cp;
+      cs.start(cu, b0, b1, p.max_ctx, sl, u);
+      cp.start(cu, b0, b1, p.max_ctx, sl, u);
+      int gs = 0, gp = 0;
+      bool s_part = false, ok = true;      // s_part: S_gs's score-only part is issued
+      uint64_t t_stall = 0;
       uint32_t idle = 0;
-      while (ok && jp < nch) {
+      while (ok && !cp.done) {
         bool progress = false;
-        if (js < nch && js < jp + NSLOT) {
-          const int st = js % NSTAGE, sl = js % NSLOT;
-          const uint32_t par = (js / NSTAGE) & 1;
-          const uint32_t d = tbase + TM_S + sl * NT;
+        if (!cs.done && gs < gp + NSLOT) {
+          const int st = gs % NSTAGE, sls = gs % NSLOT;
+          const uint32_t par = (gs / NSTAGE) & 1;
+          const uint32_t d = tbase + TM_S + sls * NT;
           const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
-          if (!s_part && mbar_test(&ca_full[st], par)) {
+          if (!s_part &&
+              (cs.j != 0 || (mbar_test(&q_full, cs.kk & 1) && mbar_test(&qt_full, cs.kk & 1))) &&
+              mbar_test(&ca_full[st], par)) {
             tc_fence_after();
             for (int i = 0; i < SO_BOXES; ++i) s_box(d, dc, score_only_box(rank, i), i == 0);
             mma_commit(&ca_empty[st]);
@@ -265,35 +400,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           if (s_part && mbar_test(&cb_full[st], par)) {
             tc_fence_after();
             for (int i = 0; i < V_BOXES; ++i) s_box(d, dc, 4 * (int)rank + i, false);
-            mma_commit(&s_full[sl]);
+            mma_commit(&s_full[sls]);
+            if (cs.j == cs.s.nch - 1) mma_commit(&q_free);
             s_part = false;
-            ++js;
+            ++gs;
+            cs.next(cu, b0, b1, p.max_ctx, sl, u);
             progress = true;
           }
         }
-        if (jp < js) {
-          const int st = jp % NSTAGE, sl = jp % NSLOT;
-          if (mbar_test(&p_full[sl], (jp / NSLOT) & 1)) {
+        if (gp < gs) {
+          const int st = gp % NSTAGE, slp = gp % NSLOT;
+          if (mbar_test(&p_full[slp], (gp / NSLOT) & 1) &&
+              (cp.j != 0 || cp.kk == 0 || mbar_test(&o_free, (cp.kk - 1) & 1))) {
             tc_fence_after();
             const uint64_t dv =
                 desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE + (dim0 / 64) * CBOX), CBOX);
 #pragma unroll
             for (int k = 0; k < NT / 16; ++k)
-              mma_bf16_ts(tbase + TM_O, tbase + TM_S + sl * NT + k * 8,
-                          dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (jp | k) != 0);
+              mma_bf16_ts(tbase + TM_O, tbase + TM_S + slp * NT + k * 8,
+                          dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (cp.j | k) != 0);
             mma_commit(&cb_empty[st]);
-            mma_commit(&pv_done[jp & 1]);
-            if (jp == nch - 1) mma_commit(&o_done);
-            ++jp;
+            mma_commit(&pv_done[gp & 1]);
+            if (cp.j == cp.s.nch - 1) mma_commit(&o_done);
+            ++gp;
+            cp.next(cu, b0, b1, p.max_ctx, sl, u);
             progress = true;
           }
         }
         if (progress) {
           idle = 0;
         } else if ((++idle & 63u) == 0) {   // bounded like every other wait
+          const uint64_t now = globaltimer();
+          if (idle == 64) t_stall = now;     // this stall began
           if (*abort_v) {
             ok = false;
-          } else if (globaltimer() - t_start > kWaitNs) {
+          } else if (now - t_stall > kWaitNs) {
             *abort_v = 1;
             atomicOr(p.status, kStatusTimeout);
             ok = false;
@@ -302,161 +443,244 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (sm_wg >= 0) {
-    // ---------------- softmax (thread = head): group g takes chunks g, g + 2,
-    // ... (always score slot g).  The reference max of every row passes from
-    // one group to the other through shared memory; each group keeps the row
-    // sum of its own chunks, relative to its last reference.
+    // ---------------- softmax (thread = head): group g takes the chunks of
+    // its parity in the unit's chunk sequence (score slot g).  The reference
+    // max of every row passes from one group to the other through shared
+    // memory; each group keeps the row sum of its own chunks, relative to its
+    // last reference.  Per segment, group 1 first stores the query's TMEM
+    // part, group 0 finally merges both groups' sums and writes the result.
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int head = h0 + r;
     const bool head_ok = head < p.h;
-    if (sm_wg == 0) {   // query latent dims [0, 256) of this head into TMEM (A operand)
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)b * p.h + head) * R);
-#pragma unroll 1
-      for (int part = 0; part < 4; ++part) {
-        uint32_t q[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = head_ok ? src[part * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
-          q[4 * c] = v.x;
-          q[4 * c + 1] = v.y;
-          q[4 * c + 2] = v.z;
-          q[4 * c + 3] = v.w;
-        }
-        tmem_st32(tbase + lane_off + TM_Q + part * 32, q);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qt_full);
-    }
-    float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = sm_wg; j < nch; j += 2) {
-      const int sl = j % NSLOT, xs = j & 1;
-      if (!warp_wait(&s_full[sl], (j / NSLOT) & 1, abort_v, p.status)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tbase + lane_off + TM_S + sl * NT, sr[0]);
-      tmem_ld32(tbase + lane_off + TM_S + sl * NT + 32, sr[1]);
-      tmem_wait_ld();
-      float s[NT];
-#pragma unroll
-      for (int i = 0; i < NT; ++i) s[i] = __uint_as_float(sr[i >> 5][i & 31]);
-      // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
-      const int lo = j * NT - (chunk_base(n, t0, j) - t0);
-      const int hi = tcount - (chunk_base(n, t0, j) - t0);
-      // Raw scores; the (positive) scale is folded into the exp argument.
-      if (lo > 0 || hi < NT) {       // first / last chunk of the split only
-#pragma unroll
-        for (int i = 0; i < NT; ++i)
-          if (i < lo || i >= hi) s[i] = -INFINITY;
-      }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int i = 0; i < NT; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], s[i], s[i + 1]);
-      const float cmax = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * p.scale_log2;
-      // reference of chunk j-1, left by the other group
-      float m_prev = -INFINITY;
-      if (j > 0) {
-        if (!warp_wait(&ref_ready[xs ^ 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        m_prev = m_hand[xs ^ 1][r];
-      }
-      // lazy rescaling: a new reference only when the max grew by > 2^8
-      const bool grow = cmax > m_prev + kRescaleLog2;     // always at j = 0
-      const float m_new = grow ? cmax : m_prev;
-      m_hand[xs][r] = m_new;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ref_ready[xs]);
-      if (m_new != m_ref) {          // this group's sum, moved to the new reference
-        l *= ex2(m_ref - m_new);
-        m_ref = m_new;
-      }
-      const float neg_m = -m_ref;
-      float ls[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
-      uint32_t w[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        float a0, a1;
-        fma2(a0, a1, s[2 * e], s[2 * e + 1], p.scale_log2, p.scale_log2, neg_m, neg_m);
-        const float p0 = ex2(a0);
-        const float p1 = ex2(a1);
-        add2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
-        w[e] = pack_bf16(p0, p1);
-      }
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      // O holds the sum through chunk j-1 at reference m_prev: rescale it
-      // when this chunk moved the reference (PV_{j-1} must be complete).
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        const float alpha = ex2(m_prev - m_new);
-        if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+    SegCursor c;
+    c.start(cu, b0, b1, p.max_ctx, sl, u);
+    for (int g0 = 0; !c.done; c.next_seg(cu, b0, b1, p.max_ctx, sl, u)) {
+      const Seg s = c.s;
+      const int kk = c.kk;
+      if (sm_wg == 1 && ok) {   // query latent dims [0, 256) of this head into TMEM
+        if (kk > 0 && !warp_wait(&q_free, (kk - 1) & 1, abort_v, p.status)) ok = false;
+        if (ok) {
+          const uint4* src =
+              reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)s.b * p.h + head) * R);
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tbase + lane_off + TM_O + c * 32, o);
-          tmem_wait_ld();
+          for (int part = 0; part < 4; ++part) {
+            uint32_t q[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tbase + lane_off + TM_O + c * 32, o);
+            for (int cc = 0; cc < 8; ++cc) {
+              const uint4 v = head_ok ? src[part * 8 + cc] : make_uint4(0u, 0u, 0u, 0u);
+              q[4 * cc] = v.x;
+              q[4 * cc + 1] = v.y;
+              q[4 * cc + 2] = v.z;
+              q[4 * cc + 3] = v.w;
+            }
+            tmem_st32(tbase + lane_off + TM_Q + part * 32, q);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&qt_full);
         }
       }
-      // P_j over the first half of S_j's slot (S_j is in registers already)
-      tmem_st32(tbase + lane_off + TM_S + sl * NT, w);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sl]);
-    }
-    // Row sum of the split: both groups' sums at the last chunk's reference
-    // (references never decrease, so that is the larger of the two).  Group 1
-    // hands over through m_hand[1] only once group 0 no longer reads it: the
-    // final barrier below orders the two.
-    if (sm_wg == 1) {
-      named_barrier_sync(1, 256);              // group 0 has left its loop
-      m_hand[1][r] = m_ref;
-      m_hand[0][r] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&fin);
-    } else {
-      named_barrier_sync(1, 256);
-      if (ok && warp_wait(&fin, 0, abort_v, p.status) &&
-          warp_wait(&o_done, 0, abort_v, p.status)) {
-        const float m1 = m_hand[1][r], l1 = m_hand[0][r];
-        const float m_last = fmaxf(m_ref, m1);
-        const float l_tot = l * ex2(m_ref - m_last) + (l1 > 0.f ? l1 * ex2(m1 - m_last) : 0.f);
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; ok && j < s.nch; ++j) {
+        const int g = g0 + j;
+        if ((g & 1) != sm_wg) continue;
+        const int sls = g % NSLOT, xs = g & 1;
+        if (!warp_wait(&s_full[sls], (g / NSLOT) & 1, abort_v, p.status)) { ok = false; break; }
         tc_fence_after();
-        const int64_t part = ((int64_t)b * p.max_splits + sp) * p.h + head;
-        const float inv = 1.f / l_tot;
-        float* dst = p.part_o + part * R + dim0;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tbase + lane_off + TM_O + c * 32, o);
-          tmem_wait_ld();
-          if (head_ok) {
+        uint32_t sr[2][32];
+        tmem_ld32(tbase + lane_off + TM_S + sls * NT, sr[0]);
+        tmem_ld32(tbase + lane_off + TM_S + sls * NT + 32, sr[1]);
+        tmem_wait_ld();
+        float sv[NT];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              st_global_v4(dst + c * 32 + i, __float_as_uint(__uint_as_float(o[i]) * inv),
-                           __float_as_uint(__uint_as_float(o[i + 1]) * inv),
-                           __float_as_uint(__uint_as_float(o[i + 2]) * inv),
-                           __float_as_uint(__uint_as_float(o[i + 3]) * inv));
+        for (int i = 0; i < NT; ++i) sv[i] = __uint_as_float(sr[i >> 5][i & 31]);
+        // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
+        const int base = chunk_base(s.n, s.t0, j) - s.t0;
+        const int lo = j * NT - base, hi = s.tcount - base;
+        // Raw scores; the (positive) scale is folded into the exp argument.
+        if (lo > 0 || hi < NT) {       // first / last chunk of the segment only
+#pragma unroll
+          for (int i = 0; i < NT; ++i)
+            if (i < lo || i >= hi) sv[i] = -INFINITY;
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < NT; i += 2)
+          mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], sv[i], sv[i + 1]);
+        const float cmax = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+        // reference of chunk g-1, left by the other group (each thread reads
+        // its row before it overwrites it).  The wait also keeps the hand-over
+        // in order across segments, where the reference itself starts afresh.
+        float m_prev = -INFINITY;
+        if (g > 0) {
+          if (!warp_wait(&ref_ready[xs ^ 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          if (j > 0) m_prev = m_hand[r];
+        }
+        // lazy rescaling: a new reference only when the max grew by > 2^8
+        const bool grow = cmax > m_prev + kRescaleLog2;     // always at j = 0
+        const float m_new = grow ? cmax : m_prev;
+        m_hand[r] = m_new;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ref_ready[xs]);
+        if (m_new != m_ref) {          // this group's sum, moved to the new reference
+          l = l > 0.f ? l * ex2(m_ref - m_new) : 0.f;
+          m_ref = m_new;
+        }
+        const float neg_m = -m_ref;
+        float ls[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float a0, a1;
+          fma2(a0, a1, sv[2 * e], sv[2 * e + 1], p.scale_log2, p.scale_log2, neg_m, neg_m);
+          const float p0 = ex2(a0);
+          const float p1 = ex2(a1);
+          add2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
+          w[e] = pack_bf16(p0, p1);
+        }
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        // O holds the segment's sum through chunk j-1 at reference m_prev:
+        // rescale it when this chunk moved the reference (PV_{g-1} must be
+        // complete).
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          const float alpha = ex2(m_prev - m_new);
+          if (!warp_wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tbase + lane_off + TM_O + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tbase + lane_off + TM_O + cc * 32, o);
           }
         }
-        if (rank == 0 && head_ok)
-          p.part_lse[part] = (m_last + __log2f(l_tot)) * 0.6931471805599453f;
+        // P_g over the first half of S_g's slot (S_g is in registers already)
+        tmem_st32(tbase + lane_off + TM_S + sls * NT, w);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sls]);
+      }
+      g0 += s.nch;
+      // Segment end.  Both groups' sums at the last chunk's reference
+      // (references never decrease, so that is the larger of the two).
+      // Group 1 hands over through fin_*, once group 0 has finished the
+      // previous segment (o_free), which it does only after reading them.
+      // Both groups pass one barrier per segment, also after a failed wait.
+      if (sm_wg == 1) {
+        if (ok && kk > 0 && !warp_wait(&o_free, (kk - 1) & 1, abort_v, p.status)) ok = false;
+        fin_m[r] = m_ref;
+        fin_l[r] = l;
+        named_barrier_sync(1, 256);
+      } else {
+        named_barrier_sync(1, 256);
+        if (ok && !warp_wait(&o_done, kk & 1, abort_v, p.status)) ok = false;
+        if (ok) {
+          const float m1 = fin_m[r], l1 = fin_l[r];
+          const float m_last = fmaxf(m_ref, m1);
+          const float l_tot = (l > 0.f ? l * ex2(m_ref - m_last) : 0.f) +
+                              (l1 > 0.f ? l1 * ex2(m1 - m_last) : 0.f);
+          const float inv = 1.f / l_tot;
+          tc_fence_after();
+          // This warp's 32 rows go out through the query buffer (free: every
+          // S of the segment has completed) and TMA stores, 32 x 64 bf16 or
+          // 32 x 32 fp32 per box; a warp whose rows straddle the head count
+          // stores directly.
+          const int row0 = h0 + quad * 32;
+          const bool tma_rows = row0 + 32 <= p.h;
+          const uint32_t stg = smem_u32(smem + OFF_Q) + quad * 2 * EPI_BOX;
+          auto stage = [&](int i, const uint32_t (&v)[32]) -> uint32_t {
+            const uint32_t sb = stg + (i & 1) * EPI_BOX;
+            if (i >= 2) {             // the store issued from this box two boxes ago
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              st_shared_v4(sb + lane * 128 + ((k ^ (lane & 7)) << 4), v[4 * k], v[4 * k + 1],
+                           v[4 * k + 2], v[4 * k + 3]);
+            fence_proxy_async();
+            __syncwarp();
+            return sb;
+          };
+          if (s.whole) {           // the sequence's attention output, final
+            __nv_bfloat16* dst = p.o_lat + ((int64_t)s.b * p.h + head) * R + dim0;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t w[32];
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                uint32_t o[32];
+                tmem_ld32(tbase + lane_off + TM_O + cc * 64 + half * 32, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  w[half * 16 + i] = pack_bf16(__uint_as_float(o[2 * i]) * inv,
+                                               __uint_as_float(o[2 * i + 1]) * inv);
+              }
+              if (tma_rows) {
+                const uint32_t sb = stage(cc, w);
+                if (lane == 0) {
+                  tma_store_2d(&tmOL, sb, dim0 + cc * 64, s.b * p.h + row0);
+                  bulk_commit_group();
+                }
+              } else if (head_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                  st_global_v4(dst + cc * 64 + 2 * i, w[i], w[i + 1], w[i + 2], w[i + 3]);
+              }
+            }
+          } else {                 // a partial (o, lse) for the combine kernel
+            const int64_t part = (int64_t)s.slot * p.h + head;
+            float* dst = p.part_o + part * R + dim0;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(tbase + lane_off + TM_O + cc * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv);
+              if (tma_rows) {
+                const uint32_t sb = stage(cc, o);
+                if (lane == 0) {       // fp32 columns as bf16 pairs
+                  tma_store_2d(&tmPO, sb, 2 * (dim0 + cc * 32), s.slot * p.h + row0);
+                  bulk_commit_group();
+                }
+              } else if (head_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                  st_global_v4(dst + cc * 32 + i, o[i], o[i + 1], o[i + 2], o[i + 3]);
+              }
+            }
+            if (rank == 0 && head_ok)
+              p.part_lse[part] = (m_last + __log2f(l_tot)) * 0.6931471805599453f;
+          }
+          // the query buffer is read out before the next segment's query lands
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          // O may be overwritten by the next segment's first PV
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_free);
+        }
       }
     }
   }
+  if (sm_wg == 0 && lane == 0) bulk_wait_group<0>();   // epilogue stores done before exit
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -466,24 +690,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// D3: o_lat[b,h] = sum_s w_s part_o[b,s,h] with w_s = exp(lse_s - max) / sum,
-// one block per (sequence, head), 4 latent columns per thread.
+// D3: o_lat[b,h] = sum_s w_s part_o[s,h] over the partial slots of sequence b
+// (w_s = exp(lse_s - max) / sum), one block per (sequence, head), 4 latent
+// columns per thread.  A sequence inside one unit's slice was written by D2
+// itself; an invalid one (length outside [1, max_ctx]) is reported and
+// zeroed.
 __global__ void __launch_bounds__(128)
     combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                   __nv_bfloat16* __restrict__ o_lat, int h, int max_splits) {
+                   __nv_bfloat16* __restrict__ o_lat, const int32_t* __restrict__ cu, int B,
+                   int max_ctx, int h, int n_units, int min_len, uint32_t* status) {
   const int b = blockIdx.x / h, hh = blockIdx.x % h;
   const int c = threadIdx.x * 4;
-  const float* lse = part_lse + (int64_t)b * max_splits * h + hh;
+  __nv_bfloat16* dst = o_lat + ((int64_t)b * h + hh) * R + c;
+  const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
+  const int64_t T = min(max((int64_t)cu[B] - c0, (int64_t)0), (int64_t)B * max_ctx);
+  if (ce - cb < 1 || ce - cb > max_ctx || cb < 0 || ce > T) {
+    if (hh == 0 && threadIdx.x == 0) atomicOr(status, kStatusBadCtx);
+    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+    return;
+  }
+  const int64_t L = max((T + n_units - 1) / n_units, (int64_t)min_len);
+  const int u0 = (int)(cb / L), u1 = (int)((ce - 1) / L);
+  if (u0 == u1) return;
   float mx = -INFINITY;
-  for (int s = 0; s < max_splits; ++s) mx = fmaxf(mx, lse[(int64_t)s * h]);
+  for (int uu = u0; uu <= u1; ++uu) {
+    const int slot = 2 * uu + (cb > (int64_t)uu * L ? 1 : 0);
+    mx = fmaxf(mx, part_lse[(int64_t)slot * h + hh]);
+  }
   float den = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-  for (int s = 0; s < max_splits; ++s) {
-    const float l = lse[(int64_t)s * h];
+  for (int uu = u0; uu <= u1; ++uu) {
+    const int slot = 2 * uu + (cb > (int64_t)uu * L ? 1 : 0);
+    const float l = part_lse[(int64_t)slot * h + hh];
     if (l == -INFINITY) continue;
     const float w = __expf(l - mx);
-    const float4 v = *reinterpret_cast<const float4*>(
-        part_o + (((int64_t)b * max_splits + s) * h + hh) * R + c);
+    const float4 v =
+        *reinterpret_cast<const float4*>(part_o + ((int64_t)slot * h + hh) * R + c);
     den += w;
     a0 = fmaf(w, v.x, a0);
     a1 = fmaf(w, v.y, a1);
@@ -491,7 +732,6 @@ __global__ void __launch_bounds__(128)
     a3 = fmaf(w, v.w, a3);
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  __nv_bfloat16* dst = o_lat + ((int64_t)b * h + hh) * R + c;
   *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(a0 * inv, a1 * inv),
                                               pack_bf16(a2 * inv, a3 * inv));
 }
@@ -503,7 +743,7 @@ bool tc_decode_supported(const mla_config& c) {
          c.qk_nope_head_dim % 8 == 0 && c.v_head_dim % 8 == 0;
 }
 
-int tc_decode_split_tokens() { return 4096; }
+int tc_decode_min_slice() { return 512; }
 
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e;
@@ -536,31 +776,43 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
     const uint64_t cdims[2] = {(uint64_t)W, (uint64_t)a.B * (uint64_t)a.max_ctx};
     const uint64_t cstr[1] = {(uint64_t)W * 2};
     if (!encode_tmap(&tmC, a.cache, 2, cdims, cstr, cbox)) return cudaErrorInvalidValue;
+    // epilogue stores: fp32 partials (as bf16 pairs) and the bf16 latent output,
+    // 32 rows x 128 bytes per box
+    CUtensorMap tmPO, tmOL;
+    const uint32_t obox[2] = {64, 32};
+    const uint64_t podims[2] = {(uint64_t)2 * R, (uint64_t)2 * a.n_units * a.h};
+    const uint64_t postr[1] = {(uint64_t)R * 4};
+    if (!encode_tmap(&tmPO, a.part_o, 2, podims, postr, obox)) return cudaErrorInvalidValue;
+    const uint64_t oldims[2] = {(uint64_t)R, (uint64_t)a.B * a.h};
+    const uint64_t olstr[1] = {(uint64_t)R * 2};
+    if (!encode_tmap(&tmOL, a.o_lat, 2, oldims, olstr, obox)) return cudaErrorInvalidValue;
     DecTcParams p{};
     p.cu_ctx = a.cu_ctx;
     p.q_lat = reinterpret_cast<const __nv_bfloat16*>(a.q_lat);
     p.B = a.B;
     p.h = a.h;
     p.max_ctx = a.max_ctx;
-    p.split_tokens = a.split_tokens;
-    p.max_splits = a.max_splits;
+    p.n_units = a.n_units;
+    p.min_len = a.min_len;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.part_o = a.part_o;
     p.part_lse = a.part_lse;
+    p.o_lat = reinterpret_cast<__nv_bfloat16*>(a.o_lat);
     p.status = a.status;
     static std::atomic<uint64_t> smem_set{0};
     {
       const cudaError_t ea = set_dynamic_smem((const void*)latent_attn_kernel, SMEM_BYTES, smem_set);
       if (ea != cudaSuccess) return ea;
     }
-    dim3 grid(2 * a.B * a.max_splits, 1, (a.h + 127) / 128);
-    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, p);
+    dim3 grid(2 * a.n_units, 1, (a.h + 127) / 128);
+    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, tmPO, tmOL, p);
     count_launches();
   }
   stage_event(2, st);
   // D3
   combine_kernel<<<a.B * a.h, R / 4, 0, st>>>(a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat,
-                                              a.h, a.max_splits);
+                                              a.cu_ctx, a.B, a.max_ctx, a.h, a.n_units,
+                                              a.min_len, a.status);
   count_launches();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -110,10 +110,11 @@ struct DecodeArgs {
   const int32_t* cu_ctx;
   int B, max_ctx, h, dn, dr, dv, r;
   float scale;
-  int split_tokens, max_splits;
+  int split_tokens, max_splits;   // SIMT path: tokens per split, splits per sequence
+  int n_units, min_len;           // tensor-core path: CTA pairs, shortest slice
   void* q_lat;          // [B, h, r + dr]
-  float* part_o;        // [B, max_splits, h, r]
-  float* part_lse;      // [B, max_splits, h]
+  float* part_o;        // SIMT [B, max_splits, h, r]; tensor cores [2 n_units, h, r]
+  float* part_lse;      // SIMT [B, max_splits, h];    tensor cores [2 n_units, h]
   void* o_lat;          // [B, h, r]
   void* o;              // [B, h, dv]
   uint32_t* status;
@@ -160,5 +161,7 @@ cudaError_t launch_latent_finalize(int dtype, const void* ckv,
                                    int dr, float eps, void* cache,
                                    cudaStream_t st, int T = 1, int dst_T = 1, int dst_off = 0);
 cudaError_t launch_decode_simt(int dtype, const DecodeArgs& a, cudaStream_t st);
+// Smallest workspace mla_decode_absorbed runs with (one SM pair on tensor cores).
+size_t decode_min_workspace(const mla_config& c, int B, int max_ctx);
 
 }  // namespace mla

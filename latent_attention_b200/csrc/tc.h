@@ -15,7 +15,8 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status);
 cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st);
 bool tc_decode_supported(const mla_config& c);
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st);
-// Tokens per split of the tensor-core decode (a multiple of its 64-token chunk).
-int tc_decode_split_tokens();
+// Shortest slice of the token stream one CTA pair of the tensor-core decode
+// takes (tokens).
+int tc_decode_min_slice();
 
 }  // namespace mla

@@ -106,9 +106,18 @@ def test_workspace_sizes_are_host_logic(lib):
     cfg3 = WORKLOADS["directq_prefill"].cfg
     _, lay3 = mla_prefill_workspace_size(cfg3, 4, 8192)
     assert lay3["q_a"] == -1 and lay3["ssq_q"] == -1
-    nd, dl = mla_decode_workspace_size(WORKLOADS["dsv3_decode"].cfg, 64, 32768)
-    assert dl["max_splits"] * dl["split_tokens"] >= 32768
+    dcfg = WORKLOADS["dsv3_decode"].cfg
+    nd, dl = mla_decode_workspace_size(dcfg, 64, 32768)
+    # tensor cores: a slice of >= 512 tokens per SM pair, two partial slots per
+    # pair, independent of B and max_ctx (148 SMs when no device is visible)
+    assert dl["split_tokens"] == 512 and dl["max_splits"] % 2 == 0 and dl["max_splits"] > 0
+    assert dl["part_lse"] - dl["part_o"] >= dl["max_splits"] * 128 * 512 * 4
     assert nd == dl["total_bytes"]
+    nd2, dl2 = mla_decode_workspace_size(dcfg, 1, 1 << 20)
+    assert dl2["max_splits"] == dl["max_splits"] and nd2 < nd
+    # other configurations: 1024-token splits of every sequence
+    _, dl3 = mla_decode_workspace_size(WORKLOADS["tiny_f32"].cfg, 3, 4000)
+    assert dl3["split_tokens"] == 1024 and dl3["max_splits"] == 4
 
 
 def _fake(addr):

@@ -146,7 +146,7 @@ DECODE_SMALL = [
     ("tiny_f32", W["tiny_f32"].cfg, [1, 7, 64, 130], 200),
     ("bf16_dsv3dims", small_bf16(), [1, 5, 300, 2049, 77], 4096),
     ("bf16_dsv3_heads", W["dsv3_decode"].cfg, [1, 1000, 33], 1024),
-    # chunk (64-token) and split (4096-token) edges, several splits per sequence
+    # chunk (64-token) edges; sequences longer than a slice
     ("bf16_dsv3_heads_edges", W["dsv3_decode"].cfg, [63, 64, 65, 4096, 4097, 8192], 8192),
     # 96 heads (Kimi-K3 MLA): a partial 128-head tile
     ("bf16_96_heads", W["dsv3_decode"].cfg.with_(num_heads=96), [1, 128, 4100], 8192),
@@ -163,6 +163,78 @@ def test_decode_small(cuda, name, cfg, ctx, max_ctx, with_o):
     ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache,
                                  di.cu_ctx, di.w_o if with_o else None)
     assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
+
+
+def _decode_units():
+    return torch.cuda.get_device_properties(0).multi_processor_count // 2
+
+
+def test_decode_many_short_sequences(cuda):
+    """Each CTA pair's slice of the token stream holds many whole sequences:
+    the query is reloaded per sequence and the results are final at once."""
+    cfg = W["dsv3_decode"].cfg
+    rng = np.random.default_rng(11)
+    ctx = [int(v) for v in rng.integers(1, 100, size=300)]
+    di = make_decode_inputs(cfg, len(ctx), ctx, seed=5)
+    _, out = run_decode(cfg, di, 128)
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)
+    assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
+
+
+def test_decode_one_sequence_over_all_units(cuda):
+    """One long sequence crosses every slice: one partial per CTA pair."""
+    cfg = W["dsv3_decode"].cfg
+    ctx = [64 * _decode_units() * 15 + 37]
+    di = make_decode_inputs(cfg, 1, ctx, seed=6)
+    _, out = run_decode(cfg, di, ctx[0])
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)
+    assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
+
+
+def test_decode_sequences_on_slice_boundaries(cuda):
+    """Sequence starts that fall exactly on, just before and just after the
+    boundaries of the equal slices (640 tokens each here)."""
+    cfg = W["dsv3_decode"].cfg
+    L = 640
+    T = L * _decode_units()
+    ctx = [L, 2 * L, 1, L - 2, 2, 3 * L - 1, 1 + L, 64]
+    ctx.append(T - sum(ctx))
+    di = make_decode_inputs(cfg, len(ctx), ctx, seed=7)
+    _, out = run_decode(cfg, di, max(ctx))
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)
+    assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
+
+
+@pytest.mark.parametrize("units", [1, 5])
+def test_decode_smaller_workspace_uses_fewer_units(cuda, units):
+    """A workspace with the partial slots of only `units` SM pairs runs on that
+    many pairs; one byte less than one pair's layout is refused."""
+    from latent_attention_b200 import (MlaError, make_config, mla_decode_absorbed,
+                                       mla_decode_workspace_size)
+    cfg = W["dsv3_decode"].cfg
+    ctx = [3000, 17, 5000, 640]
+    B, max_ctx = len(ctx), 8192
+    di = make_decode_inputs(cfg, B, ctx, seed=8)
+    c = make_config(cfg)
+    n, lay = mla_decode_workspace_size(c, B, max_ctx)
+    slot = lay["part_lse"] - lay["part_o"]            # partial o bytes, all slots
+    per_unit = 2 * slot // lay["max_splits"]
+    lse_all = lay["o_lat"] - lay["part_lse"]
+    # the full layout minus the slots of the pairs that are dropped (each
+    # buffer rounded up to 256 bytes, so this is an upper bound)
+    drop = lay["max_splits"] // 2 - units
+    nbytes = n - drop * per_unit - (drop * lse_all) // (lay["max_splits"] // 2)
+    ws = torch.empty(nbytes + 4096, dtype=torch.uint8, device=cuda)
+    args = [t.cuda() for t in (di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)]
+    out = torch.empty(B, cfg.num_heads * cfg.v_head_dim, dtype=torch.bfloat16, device=cuda)
+    mla_decode_absorbed(c, *args, B, max_ctx, None, out, ws)
+    torch.cuda.synchronize()
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)
+    assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
+    if units == 1:
+        tiny = torch.empty(lay["part_o"] + 256, dtype=torch.uint8, device=cuda)
+        with pytest.raises(MlaError, match="MLA_ERR_WORKSPACE"):
+            mla_decode_absorbed(c, *args, B, max_ctx, None, out, tiny)
 
 
 def test_decode_full_size_sampled_sequences(cuda):

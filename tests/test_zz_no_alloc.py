@@ -39,8 +39,10 @@ def test_noalloc_matches_workspace_entry_point(cuda, with_o):
         B = len(ctx)
         args, w_o = _inputs(cfg, ctx, seed, cuda, with_o)
         H = cfg.hidden_size if with_o else cfg.num_heads * cfg.v_head_dim
+        # the full layout may exceed the array: the array's call then runs on
+        # fewer SM pairs, cut at other token positions, so the two agree to
+        # rounding
         n, _ = mla_decode_workspace_size(cfg, B, max_ctx)
-        assert n <= DECODE_NOALLOC_SCRATCH_BYTES
         ws = torch.empty(n, dtype=torch.uint8, device=cuda)
         ref = torch.empty(B, H, dtype=torch.bfloat16, device=cuda)
         got = torch.full((B, H), float("nan"), dtype=torch.bfloat16, device=cuda)
