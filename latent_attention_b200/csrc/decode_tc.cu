@@ -26,15 +26,15 @@
 // O[128, 512] in fp32 fills all 512 TMEM columns, so the two CTAs of a unit
 // split it: CTA c accumulates latent columns [256c, 256c+256) of O (256 TMEM
 // columns).  Each CTA computes the full scores S = Q C^T over all 576 cached
-// dims itself -- the query's latent dims [0, 256) sit in TMEM (A operand from
-// tensor memory, 128 columns), the rest (latent [256, 512) and rope) in
-// shared memory -- so the two CTAs need no partial-score exchange and run the
-// identical online softmax.  Each CTA TMA-loads every 64-token chunk in full
-// (9 boxes of 64 dims): the pair reads the same rows at the same time, so the
-// second read is served by L2 and every cache byte crosses HBM once.  The
-// same chunk tile is the K-major B operand of S and, for the CTA's 256 latent
-// dims, the MN-major B operand of O += P C.  P_g (bf16 pairs) is written over
-// S_g's TMEM slot.
+// dims itself -- the query's dims of the CTA's own latent half sit in TMEM (A
+// operand from tensor memory, 128 columns), the other half and the rope dims
+// in shared memory, so both CTAs issue the same work -- and the two CTAs need
+// no partial-score exchange and run the identical online softmax.  Each CTA
+// TMA-loads every 64-token chunk in full (9 boxes of 64 dims): the pair reads
+// the same rows at about the same time, so the second read is served by L2
+// and every cache byte crosses HBM once.  The same chunk tile is the K-major
+// B operand of S and, for the CTA's 256 latent dims, the MN-major B operand
+// of O += P C.  P_g (bf16 pairs) is written over S_g's TMEM slot.
 // A chunk's boxes form two groups with their own barriers: the 5 boxes only
 // the scores read are released as soon as the first part of S_g has run and
 // are refilled with chunk g+2 while softmax_g and PV_g are still to come; the
@@ -68,7 +68,6 @@ constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row widt
 constexpr int NT = 64;                           // tokens per chunk
 constexpr int QBOX = 128 * 64 * 2;               // 128 heads x 64 dims bf16
 constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
-constexpr int QT_ATOMS = 4;                      // query dims [0, 256) in TMEM
 constexpr int QS_ATOMS = 5;                      // query dims [256, 576) in shared memory
 constexpr int C_ATOMS = 9;                       // a chunk's 576 dims
 constexpr int NSTAGE = 2;                        // chunk ring
@@ -82,7 +81,8 @@ constexpr int PREFETCH = 4;                              // chunks prefetched to
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
 // TMEM: score slots [0, 128) (64 columns each; P_j over the first 32 of slot
-// j % 2), O [128, 384), query dims [0, 256) as bf16 pairs [384, 512).
+// j % 2), O [128, 384), the query's latent dims [256c, 256c + 256) of CTA c
+// as bf16 pairs [384, 512).
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_Q = 384;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int SO_BOXES = 5, V_BOXES = 4;      // score-only / value boxes of a chunk
@@ -305,8 +305,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           // the previous segment's epilogue has finished with the query buffer
           if (c.kk > 0 && !mbar_wait(&o_free, (c.kk - 1) & 1, abort_v, p.status)) break;
           mbar_arrive_expect_tx(&q_full, QS_ATOMS * QBOX);
-          for (int a = 0; a < 4; ++a)      // query latent dims [256, 512)
-            tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, 256 + 64 * a, s.b * p.h + h0, &q_full);
+          for (int a = 0; a < 4; ++a)      // the other CTA's latent half of the query
+            tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, (256 - dim0) + 64 * a, s.b * p.h + h0,
+                        &q_full);
           tma_load_2d(smem + OFF_Q + 4 * QBOX, &tmQpe, 0, s.b * p.h + h0, &q_full);
         }
         if (c.j + PREFETCH < s.nch) {
@@ -355,15 +356,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // [0, 256) from TMEM, the rest from shared memory; dc describes the
       // chunk's stage
       auto s_box = [&](uint32_t d, uint64_t dc, int a, bool first) {
-        if (a < QT_ATOMS) {
+        if (a < 8 && (a >> 2) == (int)rank) {   // this CTA's latent half: query in TMEM
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ts(d, tbase + TM_Q + a * 32 + k * 8,
+            mma_bf16_ts(d, tbase + TM_Q + (a & 3) * 32 + k * 8,
                         dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
-        } else {
+        } else {                                 // the other half and rope: shared memory
+          const int qa = a < 8 ? (a & 3) : 4;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16(d, dq + (uint64_t)(((a - QT_ATOMS) * QBOX + k * 32) >> 4),
+            mma_bf16(d, dq + (uint64_t)((qa * QBOX + k * 32) >> 4),
                      dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
         }
       };
@@ -460,11 +462,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int g0 = 0; !c.done; c.next_seg(cu, b0, b1, p.max_ctx, sl, u)) {
       const Seg s = c.s;
       const int kk = c.kk;
-      if (sm_wg == 1 && ok) {   // query latent dims [0, 256) of this head into TMEM
+      if (sm_wg == 1 && ok) {   // this CTA's latent half of the head's query into TMEM
         if (kk > 0 && !warp_wait(&q_free, (kk - 1) & 1, abort_v, p.status)) ok = false;
         if (ok) {
           const uint4* src =
-              reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)s.b * p.h + head) * R);
+              reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)s.b * p.h + head) * R + dim0);
 #pragma unroll 1
           for (int part = 0; part < 4; ++part) {
             uint32_t q[32];
