@@ -41,10 +41,10 @@
 // 4 value boxes of this CTA's latent columns are released by PV_g and read
 // last by S_{g+2}, so their load overlaps the first part of S_{g+2}.
 // Between segments the query changes: the next segment's first S waits for
-// its query (the shared-memory part is reloaded once the previous segment's
-// epilogue, which stages its TMA stores in the query buffer, is done; the
-// TMEM part once the previous segment's last S has completed), and its first
-// PV for the previous O to have been read out.
+// its query (both parts are reloaded once the previous segment's last S has
+// completed), and its first PV for the previous O to have been read out.  The
+// epilogue stages its TMA stores in the value boxes of the segment's last
+// chunk, which warp 2 refills only after the epilogue.
 // Warp roles (384 threads per CTA):
 //   warp 0     TMA: each segment's query share, score-only boxes of the chunk
 //              ring (2 stages), L2 prefetch ahead (into the next segment)
@@ -302,8 +302,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           prev_nch = s.nch;
           nx = c;                          // the next segment, prefetched near this one's end
           nx.next_seg(cu, b0, b1, p.max_ctx, sl, u);
-          // the previous segment's epilogue has finished with the query buffer
-          if (c.kk > 0 && !mbar_wait(&o_free, (c.kk - 1) & 1, abort_v, p.status)) break;
+          // the previous segment's scores no longer read the query buffer
+          if (c.kk > 0 && !mbar_wait(&q_free, (c.kk - 1) & 1, abort_v, p.status)) break;
           mbar_arrive_expect_tx(&q_full, QS_ATOMS * QBOX);
           for (int a = 0; a < 4; ++a)      // the other CTA's latent half of the query
             tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, (256 - dim0) + 64 * a, s.b * p.h + h0,
@@ -334,10 +334,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (elect_one()) {
       SegCursor c;
       c.start(cu, b0, b1, p.max_ctx, sl, u);
+      // a stage whose last chunk ended a segment also holds that segment's
+      // epilogue staging: segment ordinal, or -1
+      int staged[NSTAGE] = {-1, -1};
       for (int g = 0; !c.done; ++g) {
         const Seg& s = c.s;
         const int st = g % NSTAGE;
         if (!mbar_wait(&cb_empty[st], ((g / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+        if (staged[st] >= 0 && !mbar_wait(&o_free, staged[st] & 1, abort_v, p.status)) break;
+        staged[st] = c.j == s.nch - 1 ? c.kk : -1;
         uint8_t* sc = smem + OFF_C + st * STAGE;
         mbar_arrive_expect_tx(&cb_full[st], V_BOXES * CBOX);
         const int y = (int)s.start + chunk_base(s.n, s.t0, c.j);
@@ -598,13 +603,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                               (l1 > 0.f ? l1 * ex2(m1 - m_last) : 0.f);
           const float inv = 1.f / l_tot;
           tc_fence_after();
-          // This warp's 32 rows go out through the query buffer (free: every
-          // S of the segment has completed) and TMA stores, 32 x 64 bf16 or
+          // This warp's 32 rows go out through the value boxes of the
+          // segment's last chunk (free: its PV has completed; warp 2 refills
+          // them only after o_free) and TMA stores, 32 x 64 bf16 or
           // 32 x 32 fp32 per box; a warp whose rows straddle the head count
           // stores directly.
           const int row0 = h0 + quad * 32;
           const bool tma_rows = row0 + 32 <= p.h;
-          const uint32_t stg = smem_u32(smem + OFF_Q) + quad * 2 * EPI_BOX;
+          const int g_last = g0 - 1;
+          const uint32_t stg = smem_u32(smem + OFF_C + (g_last % NSTAGE) * STAGE) +
+                               4 * rank * CBOX + quad * 2 * EPI_BOX;
           auto stage = [&](int i, const uint32_t (&v)[32]) -> uint32_t {
             const uint32_t sb = stg + (i & 1) * EPI_BOX;
             if (i >= 2) {             // the store issued from this box two boxes ago
@@ -671,7 +679,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (rank == 0 && head_ok)
               p.part_lse[part] = (m_last + __log2f(l_tot)) * 0.6931471805599453f;
           }
-          // the query buffer is read out before the next segment's query lands
+          // the staging boxes are read out before warp 2 refills them
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
           // O may be overwritten by the next segment's first PV
