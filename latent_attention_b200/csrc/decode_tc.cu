@@ -468,22 +468,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const Seg s = c.s;
       const int kk = c.kk;
       if (sm_wg == 1 && ok) {   // this CTA's latent half of the head's query into TMEM
+        // two rounds of 16 loads (the first issued before the wait for the
+        // previous segment's last S), each stored as 64 TMEM columns
+        const uint4* src =
+            reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)s.b * p.h + head) * R + dim0);
+        uint4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = head_ok ? src[i] : make_uint4(0u, 0u, 0u, 0u);
         if (kk > 0 && !warp_wait(&q_free, (kk - 1) & 1, abort_v, p.status)) ok = false;
         if (ok) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)s.b * p.h + head) * R + dim0);
-#pragma unroll 1
-          for (int part = 0; part < 4; ++part) {
-            uint32_t q[32];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              const uint4 v = head_ok ? src[part * 8 + cc] : make_uint4(0u, 0u, 0u, 0u);
-              q[4 * cc] = v.x;
-              q[4 * cc + 1] = v.y;
-              q[4 * cc + 2] = v.z;
-              q[4 * cc + 3] = v.w;
+          for (int round = 0; round < 2; ++round) {
+            if (round == 1) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                v[i] = head_ok ? src[16 + i] : make_uint4(0u, 0u, 0u, 0u);
             }
-            tmem_st32(tbase + lane_off + TM_Q + part * 32, q);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t q[32];
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                q[4 * cc] = v[half * 8 + cc].x;
+                q[4 * cc + 1] = v[half * 8 + cc].y;
+                q[4 * cc + 2] = v[half * 8 + cc].z;
+                q[4 * cc + 3] = v[half * 8 + cc].w;
+              }
+              tmem_st32(tbase + lane_off + TM_Q + round * 64 + half * 32, q);
+            }
           }
           tmem_wait_st();
           tc_fence_before();
