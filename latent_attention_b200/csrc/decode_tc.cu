@@ -120,18 +120,26 @@ __device__ __forceinline__ int chunk_base(int n, int t0, int j) {
 }
 
 // The token stream of all sequences, concatenated in cu_ctx order, is cut
-// into equal slices of L tokens, one per CTA pair ("unit"); L is at least
-// min_len.  A unit's segment of sequence b is the part of b inside its
-// slice.  A segment that covers all of b is written to o_lat directly; any
-// other segment leaves a partial (o, lse) in slot 2u (the unit's first
-// segment) or 2u + 1 (its last), which the combine kernel merges.
+// into equal slices of L positions, one per CTA pair ("unit"); L is at least
+// min_len.  Each sequence is charged kSeqCost positions ahead of its tokens
+// (the cost of starting a segment: query loads, pipeline refill, epilogue,
+// about 4.5 chunks), so a unit whose slice holds more sequence starts takes
+// fewer tokens.  Sequence b occupies positions [vs_b, vs_b + kSeqCost + n_b)
+// with vs_b = cu_ctx[b] - cu_ctx[0] + b kSeqCost.  A unit's segment of b is
+// the part of b's tokens inside its slice.  A segment that covers all of b
+// is written to o_lat directly; any other segment leaves a partial (o, lse)
+// in slot 2u (the unit's first segment) or 2u + 1 (its last), which the
+// combine kernel merges.
+constexpr int64_t kSeqCost = 288;
+
 struct Slice {
-  int64_t r0, r1, L;   // tokens [r0, r1) of the stream, relative to cu_ctx[0]
+  int64_t r0, r1, L;   // positions [r0, r1) of the charged stream
 };
 
 __device__ __forceinline__ Slice unit_slice(const int32_t* cu, int B, int max_ctx, int u,
                                             int n_units, int min_len) {
-  const int64_t T = min(max((int64_t)cu[B] - cu[0], (int64_t)0), (int64_t)B * max_ctx);
+  const int64_t T = min(max((int64_t)cu[B] - cu[0], (int64_t)0), (int64_t)B * max_ctx) +
+                    (int64_t)B * kSeqCost;
   const int64_t L = max((T + n_units - 1) / n_units, (int64_t)min_len);
   Slice s;
   s.L = L;
@@ -140,14 +148,15 @@ __device__ __forceinline__ Slice unit_slice(const int32_t* cu, int B, int max_ct
   return s;
 }
 
-// First sequence whose tokens reach past stream position r (cu_ctx is
+// First sequence whose positions reach past position r (cu_ctx is
 // non-decreasing for valid input; any input gives an index in [0, B)).
 __device__ __forceinline__ int seq_at(const int32_t* cu, int B, int64_t r) {
   int lo = 0, hi = B - 1;
   const int64_t c0 = cu[0];
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    if ((int64_t)cu[mid + 1] - c0 <= r) lo = mid + 1; else hi = mid;
+    if ((int64_t)cu[mid + 1] - c0 + (int64_t)(mid + 1) * kSeqCost <= r) lo = mid + 1;
+    else hi = mid;
   }
   return lo;
 }
@@ -167,14 +176,15 @@ __device__ __forceinline__ Seg seg_info(const int32_t* cu, int b, int max_ctx, c
   const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
   s.start = cu[b];
   const int64_t n = ce - cb;
-  const int64_t s0 = max(sl.r0, cb), s1 = min(sl.r1, ce);
+  const int64_t vs = cb + (int64_t)b * kSeqCost, v0 = vs + kSeqCost;   // charge, tokens
+  const int64_t s0 = max(sl.r0, v0), s1 = min(sl.r1, v0 + n);
   s.n = (int)min(max(n, (int64_t)0), (int64_t)max_ctx);
-  s.t0 = (int)max(s0 - cb, (int64_t)0);
+  s.t0 = (int)max(s0 - v0, (int64_t)0);
   s.tcount = (int)max(s1 - s0, (int64_t)0);
   if (n < 1 || n > max_ctx) s.tcount = 0;
   s.nch = (s.tcount + NT - 1) / NT;
   s.whole = s.t0 == 0 && s.tcount == n;
-  s.slot = 2 * u + (cb > sl.r0 ? 1 : 0);
+  s.slot = 2 * u + (vs > sl.r0 ? 1 : 0);
   return s;
 }
 
@@ -725,23 +735,26 @@ __global__ void __launch_bounds__(128)
   const int c = threadIdx.x * 4;
   __nv_bfloat16* dst = o_lat + ((int64_t)b * h + hh) * R + c;
   const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
-  const int64_t T = min(max((int64_t)cu[B] - c0, (int64_t)0), (int64_t)B * max_ctx);
-  if (ce - cb < 1 || ce - cb > max_ctx || cb < 0 || ce > T) {
+  const int64_t Tt = min(max((int64_t)cu[B] - c0, (int64_t)0), (int64_t)B * max_ctx);
+  if (ce - cb < 1 || ce - cb > max_ctx || cb < 0 || ce > Tt) {
     if (hh == 0 && threadIdx.x == 0) atomicOr(status, kStatusBadCtx);
     *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
     return;
   }
+  // the slices of latent_attn_kernel (unit_slice, seg_info)
+  const int64_t T = Tt + (int64_t)B * kSeqCost;
   const int64_t L = max((T + n_units - 1) / n_units, (int64_t)min_len);
-  const int u0 = (int)(cb / L), u1 = (int)((ce - 1) / L);
+  const int64_t vs = cb + (int64_t)b * kSeqCost, v0 = vs + kSeqCost;
+  const int u0 = (int)(v0 / L), u1 = (int)((v0 + (ce - cb) - 1) / L);
   if (u0 == u1) return;
   float mx = -INFINITY;
   for (int uu = u0; uu <= u1; ++uu) {
-    const int slot = 2 * uu + (cb > (int64_t)uu * L ? 1 : 0);
+    const int slot = 2 * uu + (vs > (int64_t)uu * L ? 1 : 0);
     mx = fmaxf(mx, part_lse[(int64_t)slot * h + hh]);
   }
   float den = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   for (int uu = u0; uu <= u1; ++uu) {
-    const int slot = 2 * uu + (cb > (int64_t)uu * L ? 1 : 0);
+    const int slot = 2 * uu + (vs > (int64_t)uu * L ? 1 : 0);
     const float l = part_lse[(int64_t)slot * h + hh];
     if (l == -INFINITY) continue;
     const float w = __expf(l - mx);

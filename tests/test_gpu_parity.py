@@ -192,13 +192,19 @@ def test_decode_one_sequence_over_all_units(cuda):
 
 
 def test_decode_sequences_on_slice_boundaries(cuda):
-    """Sequence starts that fall exactly on, just before and just after the
-    boundaries of the equal slices (640 tokens each here)."""
+    """Sequences around the boundaries of the equal slices (1280 positions
+    each here; every sequence is charged 288 positions before its tokens):
+    one ending on a boundary, one whose tokens start on a boundary, one whose
+    charge straddles a boundary, a one-token one, and one long sequence."""
     cfg = W["dsv3_decode"].cfg
-    L = 640
-    T = L * _decode_units()
-    ctx = [L, 2 * L, 1, L - 2, 2, 3 * L - 1, 1 + L, 64]
-    ctx.append(T - sum(ctx))
+    L, C = 1280, 288
+    vend = [L, 3 * L - C, 3 * L + 1, 4 * L - 111, 4 * L + C - 111 + 64]
+    ctx, pos = [], 0
+    for e in vend:
+        ctx.append(e - pos - C)
+        pos = e
+    ctx.append(L * _decode_units() - pos - C)
+    assert min(ctx) >= 1
     di = make_decode_inputs(cfg, len(ctx), ctx, seed=7)
     _, out = run_decode(cfg, di, max(ctx))
     ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx)
