@@ -246,7 +246,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int j = 0; j < my_nkv; ++j) {
       // S_X(j) completion also implies PV_X(j-1) completion (in-order MMAs,
       // and S_X(j) was issued after PV_X(j-1) completed)
-      if (!warp_wait(&s_full[x], j & 1, abort_v, p.status)) { ok = false; break; }
+      if (ok && !warp_wait(&s_full[x], j & 1, abort_v, p.status)) ok = false;
+      if (!ok) {   // after a failed wait: the halves' barriers stay paired
+        named_barrier_sync(1 + x, 256);
+        continue;
+      }
       tc_fence_after();
       uint32_t sr[2][32];
       tmem_ld32(tS + hf * 64, sr[0]);
@@ -315,8 +319,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    // row sum of both halves; the barrier also keeps the two halves' loops in
-    // step on the exit path
+    // row sum of both halves (each half passes my_nkv + 1 barriers on every
+    // path)
     l_half[x][hf][r] = l;
     named_barrier_sync(1 + x, 256);
     l = l_half[x][0][r] + l_half[x][1][r];
