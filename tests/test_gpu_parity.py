@@ -181,6 +181,22 @@ def test_decode_many_short_sequences(cuda):
     assert oracle.max_rel_err(out, ref) <= TOL[cfg.dtype]
 
 
+def test_decode_thousands_of_tiny_sequences(cuda):
+    """Dozens of one-chunk segments per CTA pair: the query reload, the
+    segment-end hand-over and the per-segment barrier phases cycle many times
+    in one launch."""
+    cfg = W["dsv3_decode"].cfg
+    rng = np.random.default_rng(12)
+    ctx = [int(v) for v in rng.integers(1, 13, size=3000)]
+    di = make_decode_inputs(cfg, len(ctx), ctx, seed=9)
+    _, out = run_decode(cfg, di, 12)
+    picks = sorted(set(range(24)) | set(range(len(ctx) - 24, len(ctx))) |
+                   set(int(v) for v in rng.integers(0, len(ctx), size=48)))
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx,
+                                 batches=picks)
+    assert oracle.max_rel_err(out[picks], ref) <= TOL[cfg.dtype]
+
+
 def test_decode_one_sequence_over_all_units(cuda):
     """One long sequence crosses every slice: one partial per CTA pair."""
     cfg = W["dsv3_decode"].cfg
