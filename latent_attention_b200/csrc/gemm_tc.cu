@@ -320,6 +320,171 @@ done:
   }
 }
 
+// ---------------------------------------------------------------------------
+// Pair variant for large non-batched GEMMs: a 2-CTA cluster computes one
+// 256 x 256 tile with cta_group::2 MMAs issued by the rank-0 CTA.  Each CTA
+// loads its 128 rows of A and its 128 of the tile's 256 B rows (32 KB per
+// k-block), so the same shared memory holds six stages instead of four and
+// covers more load latency; each CTA's TMEM holds its 128 output rows x 256
+// columns and its own epilogue warps write them.
+constexpr int BM2 = 256, STAGES2 = 6;
+constexpr int HALF_BYTES = 128 * BK * 2;                  // 16 KB
+constexpr int STAGE2_BYTES = 2 * HALF_BYTES;              // A half + B half
+constexpr int OFF_OUT2 = STAGES2 * STAGE2_BYTES;          // 192 KB
+constexpr int SMEM2_BYTES = OFF_OUT2 + 4 * 2 * OUT_BOX + 1024;
+constexpr uint32_t IDESC2 = idesc_bf16(BM2, BN);
+
+__device__ __forceinline__ void tile_coords2(const TcGemmParams& p, int t, int& s, int& m0,
+                                             int& n0) {
+  const int first = p.tiles_m * p.tiles_n[0];
+  s = (t >= first) ? 1 : 0;
+  const int local = s ? t - first : t;
+  const int tn = p.tiles_n[s], G = p.group_m;
+  const int g = local / (G * tn);
+  const int gm = min(G, p.tiles_m - g * G);
+  const int in = local - g * G * tn;
+  m0 = (g * G + in % gm) * BM2;
+  n0 = (in / gm) * BN;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmO0,
+                    const __grid_constant__ CUtensorMap tmO1,
+                    const __grid_constant__ TcGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[STAGES2], empty[STAGES2], tfull[2], tempty[2];
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  volatile int* abort_v = &abort_flag;
+  const uint32_t rank = cluster_rank();
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(&full[s], 1);       // leader: its producer's arrive + both CTAs' bytes
+      mbar_init(&empty[s], 1);      // the leader's MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);      // the leader's MMA commit
+      mbar_init(&tempty[b], 8);     // leader: the epilogue warps of both CTAs
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB0);
+    if (p.nseg > 1) tma_prefetch(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_base, TMEM_COLS);
+    tc_fence_before();
+  }
+  // both CTAs' barriers exist before either addresses the other's
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+  const int nk = (p.K + BK - 1) / BK;
+  const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);       // the leader's
+  const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+  const uint32_t peer = rank ^ 1u;
+
+  if (warp == 0) {
+    // ---------------- producer (both CTAs): this CTA's halves of each stage
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = cid; t < p.total_tiles; t += ncl) {
+        int s, m0, n0;
+        tile_coords2(p, t, s, m0, n0);
+        const CUtensorMap* tmB = s ? &tmB1 : &tmB0;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_v, p.status)) goto done;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE2_BYTES);
+          uint8_t* sa = smem + stage * STAGE2_BYTES;
+          const uint32_t fb = full0 + stage * 8;
+          tma_load_3d_pair(sa, &tmA, kb * BK, m0 + 128 * (int)rank, 0, fb);
+          tma_load_3d_pair(sa + HALF_BYTES, tmB, kb * BK, n0 + 128 * (int)rank, 0, fb);
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issue (leader only) for both CTAs
+    if (rank == 0 && elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = cid; t < p.total_tiles; t += ncl, ++local) {
+        const int buf = local & 1;
+        const uint32_t tph = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], tph ^ 1, abort_v, p.status)) goto done;
+        tc_fence_after();
+        const uint32_t d = tbase + buf * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_v, p.status)) goto done;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
+          const uint32_t sb = sa + HALF_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16_pair(d, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32),
+                          IDESC2, (kb | k) != 0);
+          const uint32_t eb = smem_u32(&empty[stage]);
+          mma_commit_pair(eb);
+          mma_commit_pair(mapa_shared(eb, peer));
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        const uint32_t tb = smem_u32(&tfull[buf]);
+        mma_commit_pair(tb);
+        mma_commit_pair(mapa_shared(tb, peer));
+      }
+    }
+  } else {
+    // ---------------- epilogue (both CTAs): this CTA's 128 rows of each tile
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t stg = smem_u32(smem + OFF_OUT2 + quad * 2 * OUT_BOX);
+    int gidx = 0;
+    int local = 0;
+    for (int t = cid; t < p.total_tiles; t += ncl, ++local) {
+      const int buf = local & 1;
+      const uint32_t tph = (local >> 1) & 1;
+      if (!warp_wait(&tfull[buf], tph, abort_v, p.status)) break;
+      tc_fence_after();
+      int s, m0, n0;
+      tile_coords2(p, t, s, m0, n0);
+      epilogue_tile(p, p.seg[s], 0, m0 + 128 * (int)rank, n0, row,
+                    tbase + ((uint32_t)(quad * 32) << 16) + buf * BN, s ? &tmO1 : &tmO0, stg,
+                    gidx);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
+    }
+    if (p.tma_store && lane == 0) bulk_wait_group<0>();   // stores done before exit
+  }
+done:
+  __syncwarp();
+  // no load, commit or arrive of either CTA addresses the other past here
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tbase, TMEM_COLS);
+  }
+}
+
 int num_sms() {
   static int n = 0;
   if (!n) {
@@ -370,11 +535,17 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
     }
     if (!encode_tmap(&tmA, a.A, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
+  // large non-batched K-major products run on CTA pairs (256-row tiles);
+  // short K (the 512-deep kv up-projection: 8 k-blocks a tile) measured
+  // faster on single CTAs
+  const bool pair = a.batch == 1 && !a.b_mn && !a.a_batch_inner && a.M >= 512 && a.K >= 1024;
+  const int bm = pair ? BM2 : BM;
+  const int b_rows = pair ? 128 : BN;     // B rows per CTA and stage
   TcGemmParams p{};
   p.M = a.M;
   p.K = a.K;
   p.nseg = a.nseg;
-  p.tiles_m = (a.M + BM - 1) / BM;
+  p.tiles_m = (a.M + bm - 1) / bm;
   p.per_batch = 0;
   for (int s = 0; s < a.nseg; ++s) {
     const int64_t n = a.seg[s].ncols;
@@ -389,7 +560,7 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
       dims[0] = a.K; dims[1] = n; dims[2] = nb;
       strides[0] = (uint64_t)a.ldb[s] * 2;
       strides[1] = a.batch > 1 ? (uint64_t)a.sB * 2 : (uint64_t)a.ldb[s] * 2 * n;
-      box[0] = BK; box[1] = BN; box[2] = 1;
+      box[0] = BK; box[1] = b_rows; box[2] = 1;
     }
     if (!encode_tmap(&tmB[s], a.Bm[s], 3, dims, strides, box)) return cudaErrorInvalidValue;
     p.seg[s] = a.seg[s];
@@ -420,11 +591,21 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   p.total_tiles = p.per_batch * a.batch;
   // long K: grouped raster (measured: o_proj, K = 16384, -0.8 %); short K keeps
   // the plain column-major order, which the 268 MB kv up-projection prefers
-  p.group_m = a.K >= 4096 ? 16 : p.tiles_m;
+  p.group_m = a.K >= 4096 ? 2048 / bm : p.tiles_m;
   p.a_batch_inner = a.a_batch_inner;
   p.b_mn = a.b_mn;
   p.sOut = a.sOut;
   p.status = status;
+  if (pair) {
+    static std::atomic<uint64_t> smem2_set{0};
+    const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc2_kernel, SMEM2_BYTES, smem2_set);
+    if (ea != cudaSuccess) return ea;
+    const int pairs = p.total_tiles < num_sms() / 2 ? p.total_tiles : num_sms() / 2;
+    gemm_tc2_kernel<<<2 * pairs, NTHREADS, SMEM2_BYTES, st>>>(tmA, tmB[0], tmB[1], tmO[0],
+                                                               tmO[1], p);
+    count_launches();
+    return cudaGetLastError();
+  }
   static std::atomic<uint64_t> smem_set{0};
   {
     const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc_kernel, SMEM_BYTES, smem_set);
