@@ -139,6 +139,22 @@ def test_prefill_full_size_sampled_rows(cuda, name):
     assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
 
 
+@pytest.mark.parametrize("name,T", [("dsv3_prefill", 777), ("dsv3_prefill", 1000),
+                                    ("directq_prefill", 1000)])
+def test_prefill_ragged_rows_on_cta_pairs(cuda, name, T):
+    """Row counts that are not a multiple of the 256-row tiles of the CTA-pair
+    projections (K >= 1024): at 777 rows the last tile's second CTA holds no
+    row, at 1000 it holds 104 of its 128."""
+    cfg = W[name].cfg
+    inp = make_prefill_inputs(cfg, 1, T, seed=4)
+    layer, out, _ = run_prefill(cfg, inp, latent=False)
+    rows = sorted(set(sample_rows(T, 24)) | {255, 256, 511, 512, 767, 768, 895, 896, T - 1})
+    rows = [r for r in rows if r < T]
+    ref = oracle.prefill(cfg, inp, rows=rows)
+    got = out[:, torch.as_tensor(rows)]
+    assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
+
+
 # --------------------------------------------------------------------------
 # Absorbed decode
 # --------------------------------------------------------------------------
