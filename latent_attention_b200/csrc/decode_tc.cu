@@ -723,22 +723,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 // D3: o_lat[b,h] = sum_s w_s part_o[s,h] over the partial slots of sequence b
-// (w_s = exp(lse_s - max) / sum), one block per (sequence, head), 4 latent
-// columns per thread.  A sequence inside one unit's slice was written by D2
-// itself; an invalid one (length outside [1, max_ctx]) is reported and
-// zeroed.
-__global__ void __launch_bounds__(128)
+// (w_s = exp(lse_s - max) / sum), one warp per (sequence, head), 8 heads per
+// block, 16 latent columns per thread.  A sequence inside one unit's slice was
+// written by D2 itself; an invalid one (length outside [1, max_ctx]) is
+// reported and zeroed.
+constexpr int kCombineHeads = 8;
+__global__ void __launch_bounds__(32 * kCombineHeads)
     combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                    __nv_bfloat16* __restrict__ o_lat, const int32_t* __restrict__ cu, int B,
                    int max_ctx, int h, int n_units, int min_len, uint32_t* status) {
-  const int b = blockIdx.x / h, hh = blockIdx.x % h;
-  const int c = threadIdx.x * 4;
-  __nv_bfloat16* dst = o_lat + ((int64_t)b * h + hh) * R + c;
+  const int hg = (h + kCombineHeads - 1) / kCombineHeads;
+  const int b = blockIdx.x / hg;
+  const int hh = (blockIdx.x % hg) * kCombineHeads + threadIdx.x / 32;
+  if (hh >= h) return;
+  const int c = (threadIdx.x % 32) * 16;
+  uint4* dst = reinterpret_cast<uint4*>(o_lat + ((int64_t)b * h + hh) * R + c);
   const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
   const int64_t Tt = min(max((int64_t)cu[B] - c0, (int64_t)0), (int64_t)B * max_ctx);
   if (ce - cb < 1 || ce - cb > max_ctx || cb < 0 || ce > Tt) {
     if (hh == 0 && threadIdx.x == 0) atomicOr(status, kStatusBadCtx);
-    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+    dst[0] = make_uint4(0u, 0u, 0u, 0u);
+    dst[1] = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
   // the slices of latent_attn_kernel (unit_slice, seg_info)
@@ -752,23 +757,32 @@ __global__ void __launch_bounds__(128)
     const int slot = 2 * uu + (vs > (int64_t)uu * L ? 1 : 0);
     mx = fmaxf(mx, part_lse[(int64_t)slot * h + hh]);
   }
-  float den = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  float den = 0.f, a[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a[i] = 0.f;
   for (int uu = u0; uu <= u1; ++uu) {
     const int slot = 2 * uu + (vs > (int64_t)uu * L ? 1 : 0);
     const float l = part_lse[(int64_t)slot * h + hh];
     if (l == -INFINITY) continue;
     const float w = __expf(l - mx);
-    const float4 v =
-        *reinterpret_cast<const float4*>(part_o + ((int64_t)slot * h + hh) * R + c);
+    const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slot * h + hh) * R + c);
     den += w;
-    a0 = fmaf(w, v.x, a0);
-    a1 = fmaf(w, v.y, a1);
-    a2 = fmaf(w, v.z, a2);
-    a3 = fmaf(w, v.w, a3);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = src[q];
+      a[4 * q] = fmaf(w, v.x, a[4 * q]);
+      a[4 * q + 1] = fmaf(w, v.y, a[4 * q + 1]);
+      a[4 * q + 2] = fmaf(w, v.z, a[4 * q + 2]);
+      a[4 * q + 3] = fmaf(w, v.w, a[4 * q + 3]);
+    }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(a0 * inv, a1 * inv),
-                                              pack_bf16(a2 * inv, a3 * inv));
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
+    dst[q] = make_uint4(pack_bf16(a[8 * q] * inv, a[8 * q + 1] * inv),
+                        pack_bf16(a[8 * q + 2] * inv, a[8 * q + 3] * inv),
+                        pack_bf16(a[8 * q + 4] * inv, a[8 * q + 5] * inv),
+                        pack_bf16(a[8 * q + 6] * inv, a[8 * q + 7] * inv));
 }
 
 }  // namespace
@@ -845,9 +859,10 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
   }
   stage_event(2, st);
   // D3
-  combine_kernel<<<a.B * a.h, R / 4, 0, st>>>(a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat,
-                                              a.cu_ctx, a.B, a.max_ctx, a.h, a.n_units,
-                                              a.min_len, a.status);
+  const int head_groups = (a.h + kCombineHeads - 1) / kCombineHeads;
+  combine_kernel<<<a.B * head_groups, 32 * kCombineHeads, 0, st>>>(
+      a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B, a.max_ctx, a.h, a.n_units,
+      a.min_len, a.status);
   count_launches();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
