@@ -19,6 +19,11 @@
 //               rope columns (see EpiSeg), bf16 stores.
 // The two TMEM accumulators let the epilogue of tile i overlap the MMAs of
 // tile i+1.  Every mbarrier wait is bounded (sm100::mbar_wait).
+//
+// Large non-batched products with K >= 1024 run on gemm_tc2_kernel instead:
+// the same roles on 2-CTA clusters with 256 x 256 tiles and cta_group::2
+// MMAs (see the comment above it), which halves each CTA's bytes per k-block
+// and so fits six stages instead of four.
 #include "sm100.cuh"
 #include "tc.h"
 
