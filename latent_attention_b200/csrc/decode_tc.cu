@@ -3,7 +3,7 @@
 // Megatron-LM MLA guide, 推理优化: each cached token keeps the compressed
 // latent [kv_compressed | k_pos_emb]; decode folds up_k (rows [0, nope) of a
 // head's block of the kv up-projection) into the query and applies up_v
-// (rows [nope, nope+v)) after attention.  Three kernels:
+// (rows [nope, nope+v)) after attention.  Four kernels:
 //
 //   D1 q_lat[b,h] = W_UK[h]^T q_nope[b,h]          batched tcgen05 GEMM (one
 //                                                   product per head, W_UK read
@@ -16,8 +16,9 @@
 //
 // D2 schedule.  The tokens of all sequences, concatenated in cu_ctx order,
 // are cut into equal slices, one per CTA pair ("unit", one pair per two
-// SMs, a single wave), so every unit has the same number of cache rows to
-// read whatever the length mix.  A unit walks the segments of its slice (the
+// SMs, a single wave), each sequence charged a fixed number of extra
+// positions for the cost of starting it (kSeqCost), so every unit has about
+// the same work whatever the length mix.  A unit walks the segments of its slice (the
 // parts of the sequences inside it) with one continuous chunk pipeline; a
 // segment covering a whole sequence writes o_lat itself, the first and last
 // segment of a slice leave a partial (o, lse) for D3.
