@@ -724,18 +724,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 // D3: o_lat[b,h] = sum_s w_s part_o[s,h] over the partial slots of sequence b
-// (w_s = exp(lse_s - max) / sum), one warp per (sequence, head), 8 heads per
-// block, 16 latent columns per thread.  A sequence inside one unit's slice was
-// written by D2 itself; an invalid one (length outside [1, max_ctx]) is
-// reported and zeroed.
-constexpr int kCombineHeads = 8;
-__global__ void __launch_bounds__(32 * kCombineHeads)
+// (w_s = exp(lse_s - max) / sum), one warp per (sequence, head), HPB heads
+// per block, 16 latent columns per thread.  A sequence inside one unit's
+// slice was written by D2 itself; an invalid one (length outside [1,
+// max_ctx]) is reported and zeroed.
+template <int HPB>
+__global__ void __launch_bounds__(32 * HPB)
     combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                    __nv_bfloat16* __restrict__ o_lat, const int32_t* __restrict__ cu, int B,
                    int max_ctx, int h, int n_units, int min_len, uint32_t* status) {
-  const int hg = (h + kCombineHeads - 1) / kCombineHeads;
+  const int hg = (h + HPB - 1) / HPB;
   const int b = blockIdx.x / hg;
-  const int hh = (blockIdx.x % hg) * kCombineHeads + threadIdx.x / 32;
+  const int hh = (blockIdx.x % hg) * HPB + threadIdx.x / 32;
   if (hh >= h) return;
   const int c = (threadIdx.x % 32) * 16;
   uint4* dst = reinterpret_cast<uint4*>(o_lat + ((int64_t)b * h + hh) * R + c);
@@ -860,10 +860,18 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
   }
   stage_event(2, st);
   // D3
-  const int head_groups = (a.h + kCombineHeads - 1) / kCombineHeads;
-  combine_kernel<<<a.B * head_groups, 32 * kCombineHeads, 0, st>>>(
-      a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B, a.max_ctx, a.h, a.n_units,
-      a.min_len, a.status);
+  // eight heads per block when the (sequence, head) pairs fill the GPU many
+  // times over (fewer, fuller blocks); one otherwise (few sequences, many
+  // partial slots each, spread over as many SMs as possible)
+  if ((int64_t)a.B * a.h >= 16LL * (2 * a.n_units)) {
+    combine_kernel<8><<<a.B * ((a.h + 7) / 8), 32 * 8, 0, st>>>(
+        a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B, a.max_ctx, a.h,
+        a.n_units, a.min_len, a.status);
+  } else {
+    combine_kernel<1><<<a.B * a.h, 32, 0, st>>>(
+        a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B, a.max_ctx, a.h,
+        a.n_units, a.min_len, a.status);
+  }
   count_launches();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
