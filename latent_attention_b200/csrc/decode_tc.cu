@@ -57,6 +57,7 @@
 // All waits are bounded; a timeout sets the device status word.
 #include <cfloat>
 
+#include "decode_slices.cuh"
 #include "sm100.cuh"
 #include "tc.h"
 
@@ -64,9 +65,9 @@ namespace mla {
 namespace {
 
 using namespace sm100;
+using namespace slices;   // NT (tokens per chunk), the slice schedule
 
 constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row width
-constexpr int NT = 64;                           // tokens per chunk
 constexpr int QBOX = 128 * 64 * 2;               // 128 heads x 64 dims bf16
 constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
 constexpr int QS_ATOMS = 5;                      // query dims [256, 576) in shared memory
@@ -119,109 +120,6 @@ __device__ __forceinline__ int chunk_base(int n, int t0, int j) {
   const int lt = t0 + j * NT;
   return n >= NT ? min(lt, n - NT) : n - NT;
 }
-
-// The token stream of all sequences, concatenated in cu_ctx order, is cut
-// into equal slices of L positions, one per CTA pair ("unit"); L is at least
-// min_len.  Each sequence is charged kSeqCost positions ahead of its tokens
-// (the cost of starting a segment: query loads, pipeline refill, epilogue,
-// about 4.5 chunks), so a unit whose slice holds more sequence starts takes
-// fewer tokens.  Sequence b occupies positions [vs_b, vs_b + kSeqCost + n_b)
-// with vs_b = cu_ctx[b] - cu_ctx[0] + b kSeqCost.  A unit's segment of b is
-// the part of b's tokens inside its slice.  A segment that covers all of b
-// is written to o_lat directly; any other segment leaves a partial (o, lse)
-// in slot 2u (the unit's first segment) or 2u + 1 (its last), which the
-// combine kernel merges.
-constexpr int64_t kSeqCost = 288;
-
-struct Slice {
-  int64_t r0, r1, L;   // positions [r0, r1) of the charged stream
-};
-
-__device__ __forceinline__ Slice unit_slice(const int32_t* cu, int B, int max_ctx, int u,
-                                            int n_units, int min_len) {
-  const int64_t T = min(max((int64_t)cu[B] - cu[0], (int64_t)0), (int64_t)B * max_ctx) +
-                    (int64_t)B * kSeqCost;
-  const int64_t L = max((T + n_units - 1) / n_units, (int64_t)min_len);
-  Slice s;
-  s.L = L;
-  s.r0 = min((int64_t)u * L, T);
-  s.r1 = min(s.r0 + L, T);
-  return s;
-}
-
-// First sequence whose positions reach past position r (cu_ctx is
-// non-decreasing for valid input; any input gives an index in [0, B)).
-__device__ __forceinline__ int seq_at(const int32_t* cu, int B, int64_t r) {
-  int lo = 0, hi = B - 1;
-  const int64_t c0 = cu[0];
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if ((int64_t)cu[mid + 1] - c0 + (int64_t)(mid + 1) * kSeqCost <= r) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
-
-struct Seg {
-  int b, n, t0, tcount, nch, slot;
-  int64_t start;       // cache row of the sequence's token 0
-  bool whole;          // the segment covers the whole sequence
-};
-
-// Segment of sequence b in the slice of unit u; nch = 0 when it is empty or
-// the sequence is invalid (the combine kernel reports those).
-__device__ __forceinline__ Seg seg_info(const int32_t* cu, int b, int max_ctx, const Slice& sl,
-                                        int u) {
-  Seg s;
-  s.b = b;
-  const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
-  s.start = cu[b];
-  const int64_t n = ce - cb;
-  const int64_t vs = cb + (int64_t)b * kSeqCost, v0 = vs + kSeqCost;   // charge, tokens
-  const int64_t s0 = max(sl.r0, v0), s1 = min(sl.r1, v0 + n);
-  s.n = (int)min(max(n, (int64_t)0), (int64_t)max_ctx);
-  s.t0 = (int)max(s0 - v0, (int64_t)0);
-  s.tcount = (int)max(s1 - s0, (int64_t)0);
-  if (n < 1 || n > max_ctx) s.tcount = 0;
-  s.nch = (s.tcount + NT - 1) / NT;
-  s.whole = s.t0 == 0 && s.tcount == n;
-  s.slot = 2 * u + (vs > sl.r0 ? 1 : 0);
-  return s;
-}
-
-// Walks the non-empty segments of a unit in order.
-struct SegCursor {
-  int k, kk;           // sequence offset from b0, ordinal among non-empty segments
-  int j;               // chunk within the segment
-  Seg s;
-  bool done;
-  __device__ __forceinline__ void seek(const int32_t* cu, int b0, int b1, int max_ctx,
-                                       const Slice& sl, int u) {
-    for (; b0 + k < b1; ++k) {
-      s = seg_info(cu, b0 + k, max_ctx, sl, u);
-      if (s.nch > 0) { done = false; return; }
-    }
-    done = true;
-  }
-  __device__ __forceinline__ void start(const int32_t* cu, int b0, int b1, int max_ctx,
-                                        const Slice& sl, int u) {
-    k = 0; kk = 0; j = 0;
-    seek(cu, b0, b1, max_ctx, sl, u);
-  }
-  __device__ __forceinline__ void next_seg(const int32_t* cu, int b0, int b1, int max_ctx,
-                                           const Slice& sl, int u) {
-    j = 0; ++k; ++kk;
-    seek(cu, b0, b1, max_ctx, sl, u);
-  }
-  // next chunk; true when it starts a new segment
-  __device__ __forceinline__ bool next(const int32_t* cu, int b0, int b1, int max_ctx,
-                                       const Slice& sl, int u) {
-    if (++j < s.nch) return false;
-    j = 0; ++k; ++kk;
-    seek(cu, b0, b1, max_ctx, sl, u);
-    return true;
-  }
-};
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -739,30 +637,23 @@ __global__ void __launch_bounds__(32 * HPB)
   if (hh >= h) return;
   const int c = (threadIdx.x % 32) * 16;
   uint4* dst = reinterpret_cast<uint4*>(o_lat + ((int64_t)b * h + hh) * R + c);
-  const int64_t c0 = cu[0], cb = (int64_t)cu[b] - c0, ce = (int64_t)cu[b + 1] - c0;
-  const int64_t Tt = min(max((int64_t)cu[B] - c0, (int64_t)0), (int64_t)B * max_ctx);
-  if (ce - cb < 1 || ce - cb > max_ctx || cb < 0 || ce > Tt) {
+  const SeqUnits su = seq_units(cu, b, B, max_ctx, n_units, min_len);
+  if (!su.valid) {
     if (hh == 0 && threadIdx.x == 0) atomicOr(status, kStatusBadCtx);
     dst[0] = make_uint4(0u, 0u, 0u, 0u);
     dst[1] = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
-  // the slices of latent_attn_kernel (unit_slice, seg_info)
-  const int64_t T = Tt + (int64_t)B * kSeqCost;
-  const int64_t L = max((T + n_units - 1) / n_units, (int64_t)min_len);
-  const int64_t vs = cb + (int64_t)b * kSeqCost, v0 = vs + kSeqCost;
-  const int u0 = (int)(v0 / L), u1 = (int)((v0 + (ce - cb) - 1) / L);
-  if (u0 == u1) return;
+  const int u0 = su.u0, u1 = su.u1;
+  if (u0 == u1) return;   // one unit covered the sequence and wrote o_lat
   float mx = -INFINITY;
-  for (int uu = u0; uu <= u1; ++uu) {
-    const int slot = 2 * uu + (vs > (int64_t)uu * L ? 1 : 0);
-    mx = fmaxf(mx, part_lse[(int64_t)slot * h + hh]);
-  }
+  for (int uu = u0; uu <= u1; ++uu)
+    mx = fmaxf(mx, part_lse[(int64_t)seq_slot(su, uu) * h + hh]);
   float den = 0.f, a[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) a[i] = 0.f;
   for (int uu = u0; uu <= u1; ++uu) {
-    const int slot = 2 * uu + (vs > (int64_t)uu * L ? 1 : 0);
+    const int slot = seq_slot(su, uu);
     const float l = part_lse[(int64_t)slot * h + hh];
     if (l == -INFINITY) continue;
     const float w = __expf(l - mx);
