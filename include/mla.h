@@ -66,7 +66,7 @@ typedef enum mla_status {
   MLA_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned              */
   MLA_ERR_DTYPE = 4,          /* cfg->dtype is not an mla_dtype                */
   MLA_ERR_WORKSPACE = 5,      /* workspace smaller than the *_workspace_size   */
-  MLA_ERR_UNSUPPORTED = 6,    /* valid MLA shape this build does not implement */
+  MLA_ERR_UNSUPPORTED = 6,    /* valid MLA shape the library does not implement */
   MLA_ERR_CUDA = 7,           /* a CUDA runtime call or launch failed          */
   MLA_ERR_DEVICE_TIMEOUT = 8  /* a bounded on-device wait gave up (reported by
                                  mla_check_device_status)                      */
