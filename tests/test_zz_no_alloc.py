@@ -58,7 +58,12 @@ def test_noalloc_rejects_oversized_requests(cuda):
     B, max_ctx = 64, 32768                        # needs far more than the array
     n, _ = mla_decode_workspace_size(cfg, B, max_ctx)
     assert n > DECODE_NOALLOC_SCRATCH_BYTES
-    t = torch.empty(16, dtype=torch.bfloat16, device=cuda)
+    h, r, dr = cfg.num_heads, cfg.kv_lora_rank, cfg.qk_rope_head_dim
+    dn, dv = cfg.qk_nope_head_dim, cfg.v_head_dim
+    bf = dict(dtype=torch.bfloat16, device=cuda)
     with pytest.raises(MlaError, match="MLA_ERR_WORKSPACE.*static array"):
-        mla_decode_absorbed_noalloc(cfg, t, t, t, t, t.view(torch.int32), B,
-                                    max_ctx, None, t)
+        mla_decode_absorbed_noalloc(
+            cfg, torch.empty(B, h, dn, **bf), torch.empty(B, h, dr, **bf),
+            torch.empty(h * (dn + dv), r, **bf), torch.empty(1, r + dr, **bf),
+            torch.zeros(B + 1, dtype=torch.int32, device=cuda), B, max_ctx, None,
+            torch.empty(B, h * dv, **bf))
