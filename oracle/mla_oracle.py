@@ -277,6 +277,17 @@ def prefill(cfg, inp, rows: Optional[Sequence[int]] = None,
 # ---------------------------------------------------------------------------
 # Chunked prefill against a cached latent
 # ---------------------------------------------------------------------------
+def _chunk_positions(T_past, T_new):
+    """Positions of the new tokens: they follow the T_past cached ones."""
+    return T_past + np.arange(T_new)
+
+
+def _chunk_latent(past, new_rows):
+    """Latent rows of every key position: the cached rows as they are (already
+    normalised and roped), then the new tokens' rows."""
+    return np.concatenate([past, new_rows], axis=1)
+
+
 def prefill_chunked(cfg, inp, past_cache, T_past: int,
                     return_parts: bool = False):
     """T_new new tokens per sequence after T_past cached ones.
@@ -317,18 +328,18 @@ def prefill_chunked(cfg, inp, past_cache, T_past: int,
         q = x @ _f64(inp.w_q).T
     q = q.reshape(B, Tn, h, dq)
     q_nope, q_pe = q[..., :dn], q[..., dn:]
+    qpos = _chunk_positions(T_past, Tn)
     if cfg.rope_type != "none":
         q_pe, kpe = _rope_columns(cfg, q_pe), _rope_columns(cfg, kpe)
         cos, sin = rope_tables(cfg, Ta)
-        cn, sn = cos[T_past:Ta], sin[T_past:Ta]
+        cn, sn = cos[qpos], sin[qpos]
         kpe = apply_rope(kpe, cn[None], sn[None])
         q_pe = apply_rope(q_pe, cn[None, :, None, :], sn[None, :, None, :])
-    latent = np.concatenate([past, np.concatenate([c_hat, kpe], -1)], axis=1)
+    latent = _chunk_latent(past, np.concatenate([c_hat, kpe], -1))
     kv = (latent[..., :r_kv] @ _f64(inp.w_kv_b).T).reshape(B, Ta, h, dn + dv)
     k_nope, v = kv[..., :dn], kv[..., dn:]
     k_pe = latent[..., r_kv:]
     o = np.empty((B, Tn, h, dv))
-    qpos = T_past + np.arange(Tn)
     mask = np.arange(Ta)[None, :] > qpos[:, None]
     for b in range(B):
         for hh in range(h):

@@ -397,6 +397,29 @@ def test_chunked_prefill_sees_all_history():
                                    rtol=1e-12, atol=1e-14)
 
 
+CHUNK_MISTAKES = {
+    # new tokens placed at positions 0.. instead of after the history (their
+    # RoPE angles and their causal mask both shift)
+    "positions_not_offset": ("_chunk_positions", lambda T_past, T_new: np.arange(T_new)),
+    # the history's latent rows lost
+    "history_zeroed": ("_chunk_latent",
+                       lambda past, new: np.concatenate([np.zeros_like(past), new], 1)),
+    # the cached latents (kv_lora_rank 8 in tiny_cfg) normalised a second
+    # time: they are stored normalised, with the gain applied
+    "history_normalised_again": ("_chunk_latent", lambda past, new: np.concatenate(
+        [np.concatenate([O.rms_norm(past[..., :8], np.ones(8), 1e-6), past[..., 8:]], -1),
+         new], 1)),
+}
+
+
+@pytest.mark.parametrize("mistake", sorted(CHUNK_MISTAKES))
+def test_planted_chunked_mistake_is_caught(monkeypatch, mistake):
+    attr, fn = CHUNK_MISTAKES[mistake]
+    monkeypatch.setattr(O, attr, fn)
+    with pytest.raises(AssertionError):
+        test_chunked_prefill_equals_full_prefill_rows("plain", 3, 4)
+
+
 # --------------------------------------------------------------------------
 # Packed (THD) prefill (Megatron 训练支持与并行策略: cu_seqlens packing)
 # --------------------------------------------------------------------------
