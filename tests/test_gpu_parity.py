@@ -303,6 +303,28 @@ def test_decode_bad_context_is_flagged(cuda):
     dec.check_status()                       # the word was cleared
 
 
+def test_decode_empty_sequence_is_flagged_and_zeroed(cuda):
+    """A sequence with no cached token has nothing to attend to: its output
+    row is zero, the status word reports it, and the sequences around it (each
+    inside one slice here) are unaffected."""
+    from latent_attention_b200 import MlaError
+    from latent_attention_b200.layer import MlaDecode
+    cfg = W["dsv3_decode"].cfg
+    di = make_decode_inputs(cfg, 3, [5, 0, 9], seed=10)
+    dec = MlaDecode(cfg, 3, 16)
+    out = torch.full((3, cfg.num_heads * cfg.v_head_dim), float("nan"), dtype=torch.bfloat16,
+                     device=cuda)
+    dec(di.q_nope.cuda(), di.q_pe.cuda(), di.w_kv_b.cuda(), di.cache.cuda(),
+        di.cu_ctx.cuda(), out)
+    torch.cuda.synchronize()
+    with pytest.raises(MlaError, match="MLA_ERR_SHAPE"):
+        dec.check_status()
+    assert torch.all(out[1] == 0)
+    ref = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache, di.cu_ctx,
+                                 batches=[0, 2])
+    assert oracle.max_rel_err(out[[0, 2]], ref) <= TOL[cfg.dtype]
+
+
 def test_bounded_wait_times_out_and_reports(cuda):
     """A device wait that nothing satisfies gives up after its bound, sets the
     status word, and leaves the context usable (failure detection without a
