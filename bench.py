@@ -62,6 +62,19 @@ def decode_work(cfg, ctx_total, B):
             "flops": flops}
 
 
+def d2_tensor_view(cfg, ctx_total, ms, peak_tflops):
+    """The latent attention kernel's tensor work as executed: both CTAs of a
+    pair compute the full scores over all kv_lora_rank + rope dims and each
+    its half of P.C, i.e. 2 (2 (r + rope)) + 2 r FLOP per token and head
+    (the algorithmic count has 2 (r + rope) + 2 r)."""
+    h, r, dr = cfg.num_heads, cfg.kv_lora_rank, cfg.qk_rope_head_dim
+    algo = ctx_total * h * (2 * (r + dr) + 2 * r)
+    executed = ctx_total * h * (2 * 2 * (r + dr) + 2 * r)
+    a = executed / (ms * 1e-3) / 1e12
+    return {"flop_executed": executed, "flop_algorithmic": algo, "achieved": a,
+            "peak": peak_tflops, "unit": "TFLOP/s", "frac": a / peak_tflops}
+
+
 def source_hash():
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "latent_attention_b200", "csrc", "*"))):
@@ -489,6 +502,8 @@ def main():
     stages = {n: roof(n, st_p[n], "tensor") for n in STAGES_P}
     stages["d2_latent_attention"] = roof("d2_latent_attention",
                                          st_d["d2_latent_attention"], "hbm")
+    stages["d2_latent_attention"]["tensor_executed"] = d2_tensor_view(
+        cfgd, ctx_total, st_d["d2_latent_attention"], peaks["bf16_sustained"])
     dominant = max(STAGES_P, key=lambda n: st_p[n])
     roofline = dict(stages[dominant], kernel=dominant,
                     peak_source=f"{peaks['source']} (bf16 sustained / HBM copy)")

@@ -1,0 +1,41 @@
+"""bench.py's work accounting, on the host: the algorithmic FLOP and byte
+counts behind ``value`` and ``roofline``, checked against counts written out
+independently for the DeepSeek-V3 workloads."""
+import bench
+from mla_inputs import WORKLOADS
+
+
+def test_prefill_flops_of_the_dsv3_workload():
+    # 2N[H r_q + r_q h 192 + H (r_kv + 64) + r_kv h 256 + h 128 H] + B h 320 T (T + 1)
+    cfg = WORKLOADS["dsv3_prefill"].cfg
+    N, H, h, T = 4096, 7168, 128, 4096
+    f = bench.prefill_stage_flops(cfg, 1, T)
+    assert f["s1_down_proj"] == 2 * N * H * (1536 + 512 + 64)
+    assert f["s3_q_proj"] == 2 * N * 1536 * h * 192
+    assert f["s4_kv_up_proj"] == 2 * N * 512 * h * 256
+    assert f["s7_attention"] == h * 320 * T * (T + 1)
+    assert f["s8_o_proj"] == 2 * N * h * 128 * H
+    assert abs(sum(f.values()) - 2.220e12) < 0.001e12
+
+
+def test_prefill_flops_direct_q():
+    cfg = WORKLOADS["directq_prefill"].cfg
+    f = bench.prefill_stage_flops(cfg, 4, 8192)
+    assert f["s1_down_proj"] == 2 * 4 * 8192 * 4096 * (512 + 64)
+    assert f["s3_q_proj"] == 2 * 4 * 8192 * 4096 * 32 * 192
+    assert abs(sum(f.values()) - 5.927e12) < 0.001e12
+
+
+def test_decode_bytes_and_executed_tensor_work():
+    cfg = WORKLOADS["dsv3_decode"].cfg
+    ctx = 1067537
+    w = bench.decode_work(cfg, ctx, 64)
+    assert w["cache_bytes"] == ctx * 576 * 2
+    assert w["bytes"] == ctx * 1152 + 128 * 256 * 512 * 2 + 64 * 128 * (192 + 128) * 2
+    v = bench.d2_tensor_view(cfg, ctx, 0.5, 1000.0)
+    # scores on both CTAs of a pair (2 x 2 x 576) plus P.C split between them
+    # (2 x 512), against the algorithmic 2 x 576 + 2 x 512 per token and head
+    assert v["flop_executed"] == ctx * 128 * 3328
+    assert v["flop_algorithmic"] == ctx * 128 * 2176
+    assert abs(v["achieved"] - ctx * 128 * 3328 / 0.5e-3 / 1e12) < 1e-9
+    assert abs(v["frac"] - v["achieved"] / 1000.0) < 1e-12
