@@ -27,6 +27,8 @@ sys.path.insert(0, ROOT)
 
 PREFILL = "dsv3_prefill"
 DECODE = "dsv3_decode"
+PREFILL_OTHERS = ["dsv3_prefill", "directq_prefill", "kimi_prefill"]
+HBM_NOMINAL_GBS = 8000.0          # the ~8 TB/s datasheet HBM3e figure
 L2_FLUSH_BYTES = 256 << 20
 STAGES_P = ["s1_down_proj", "s3_q_proj", "s4_kv_up_proj", "s7_attention",
             "s8_o_proj"]
@@ -62,17 +64,114 @@ def decode_work(cfg, ctx_total, B):
             "flops": flops}
 
 
+# Score copies the latent attention kernel computes per token and head: both
+# CTAs of an SM pair compute the full scores over all r + rope dims.
+D2_SCORE_COPIES = 2
+
+
+def d2_own_bytes(cfg, ctx_total, B):
+    """Algorithmic DRAM bytes of the latent attention kernel alone: the cache
+    rows it streams, the absorbed query it reads (q_lat and q_pe) and the
+    latent output it writes.  Partial results of sequences cut between SM
+    pairs are the schedule's overhead and are not counted; the kv
+    up-projection weights belong to the q-absorb and V-up GEMMs."""
+    h, r, dr = cfg.num_heads, cfg.kv_lora_rank, cfg.qk_rope_head_dim
+    return ctx_total * (r + dr) * 2 + B * h * (r + dr) * 2 + B * h * r * 2
+
+
 def d2_tensor_view(cfg, ctx_total, ms, peak_tflops):
-    """The latent attention kernel's tensor work as executed: both CTAs of a
-    pair compute the full scores over all kv_lora_rank + rope dims and each
-    its half of P.C, i.e. 2 (2 (r + rope)) + 2 r FLOP per token and head
-    (the algorithmic count has 2 (r + rope) + 2 r)."""
+    """The latent attention kernel's tensor work as executed: D2_SCORE_COPIES
+    x 2 (r + rope) score FLOP plus 2 r FLOP of P.C per token and head (the
+    algorithmic count has one copy of the scores)."""
     h, r, dr = cfg.num_heads, cfg.kv_lora_rank, cfg.qk_rope_head_dim
     algo = ctx_total * h * (2 * (r + dr) + 2 * r)
-    executed = ctx_total * h * (2 * 2 * (r + dr) + 2 * r)
+    executed = ctx_total * h * (D2_SCORE_COPIES * 2 * (r + dr) + 2 * r)
     a = executed / (ms * 1e-3) / 1e12
     return {"flop_executed": executed, "flop_algorithmic": algo, "achieved": a,
             "peak": peak_tflops, "unit": "TFLOP/s", "frac": a / peak_tflops}
+
+
+def roof_tensor(flops, ms, peaks, traffic=None):
+    """A tensor-core kernel against the measured burst bf16 peak: the timed
+    region lasts tens of milliseconds at the maximum SM clock, not the
+    seconds under the power cap that the sustained figure describes (kept
+    beside it as frac_sustained)."""
+    a = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": a, "peak": peaks["bf16"],
+            "unit": "TFLOP/s", "frac": a / peaks["bf16"],
+            "peak_sustained": peaks["bf16_sustained"],
+            "frac_sustained": a / peaks["bf16_sustained"], "traffic": traffic}
+
+
+def roof_hbm(nbytes, ms, peaks, traffic=None):
+    """A bandwidth-bound kernel against the measured HBM copy rate (and the
+    ~8 TB/s datasheet figure)."""
+    a = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": a / peaks["hbm"], "frac_of_8tbs": a / HBM_NOMINAL_GBS,
+            "bytes": nbytes, "traffic": traffic}
+
+
+def time_prefill_workload(wl, seed, K, Wm, flush, dev, world, set_events, tensor_roof,
+                          gpu):
+    """Time K prefill forwards of one more workload (after Wm warm-up ones),
+    the L2 flushed before each, with the library's stage events; returns its
+    throughput, stage times, the rooflines of its attention and dominant
+    kernels and the clocks sampled while it ran.  Timing is the max over
+    ranks."""
+    import torch
+    from mla_inputs import make_prefill_inputs
+    from latent_attention_b200.layer import MlaPrefill
+    cfg, B, T = wl.cfg, wl.batch, wl.seq_len
+    inp = make_prefill_inputs(cfg, B, T, seed=seed)
+    weights = {k: getattr(inp, k) for k in ("w_q_a", "g_q_a", "w_q_b", "w_q",
+                                              "w_kv_a", "g_kv_a", "w_kv_b", "w_o")}
+    pre = MlaPrefill(cfg, weights, B, T, device=dev)
+    x = inp.x.to(dev)
+    out = torch.empty(B, T, cfg.hidden_size, dtype=torch.bfloat16, device=dev)
+    del inp, weights
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [[mk() for _ in range(6)] for _ in range(K)]
+    for group in ev:
+        for e in group:
+            e.record()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu)
+    clocks.start()
+    t_begin = None
+    for i in range(Wm + K):
+        flush.zero_()
+        if i == Wm:
+            if world > 1:
+                import torch.distributed as dist
+                dist.barrier()
+            torch.cuda.synchronize()
+            t_begin = time.time()
+        set_events(ev[i - Wm] if i >= Wm else None)
+        pre(x, out=out)
+        set_events(None)
+    torch.cuda.synchronize()
+    clocks.mark(t_begin, time.time())
+    clk = clocks.stop()
+    pre.check_status()
+    ms = sum(e[0].elapsed_time(e[5]) for e in ev)
+    st = {n: sum(e[k].elapsed_time(e[k + 1]) for e in ev) / K
+          for k, n in enumerate(STAGES_P)}
+    ms = max_over_ranks([ms], world, dev)[0]
+    fl = prefill_stage_flops(cfg, B, T)
+    dominant = max(STAGES_P, key=lambda n: st[n])
+    res = {"B": B, "T": T, "hidden": cfg.hidden_size, "heads": cfg.num_heads,
+           "q_lora_rank": cfg.q_lora_rank, "rope": cfg.rope_type,
+           "ms": ms / K, "tflops": world * K * sum(fl.values()) / (ms * 1e-3) / 1e12,
+           "tokens_per_s": world * K * B * T / (ms * 1e-3),
+           "stage_ms": {k: round(v, 4) for k, v in st.items()},
+           "attention_roofline": tensor_roof(fl["s7_attention"], st["s7_attention"], None),
+           "roofline": dict(tensor_roof(fl[dominant], st[dominant], None), kernel=dominant),
+           "clocks": clk}
+    res["frac_of_peak"] = res["tflops"] / res["attention_roofline"]["peak"]
+    del pre, x, out
+    torch.cuda.empty_cache()
+    return res
 
 
 def source_hash():
@@ -489,24 +588,33 @@ def main():
     traffic = load_traffic()
     value = world * K * pflops / (pre_ms * 1e-3) / 1e12
 
-    def roof(stage, ms, bound):
-        if bound == "tensor":
-            a = fl[stage] / (ms * 1e-3) / 1e12
-            return {"bound": "tensor", "achieved": a, "peak": peaks["bf16_sustained"],
-                    "unit": "TFLOP/s", "frac": a / peaks["bf16_sustained"],
-                    "traffic": traffic.get(stage)}
-        a = dw["bytes"] / (ms * 1e-3) / 1e9
-        return {"bound": "hbm", "achieved": a, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": a / peaks["hbm"], "traffic": traffic.get(stage)}
+    def tensor_roof(flops, ms, stage):
+        return roof_tensor(flops, ms, peaks, traffic.get(stage))
 
-    stages = {n: roof(n, st_p[n], "tensor") for n in STAGES_P}
-    stages["d2_latent_attention"] = roof("d2_latent_attention",
-                                         st_d["d2_latent_attention"], "hbm")
+    def hbm_roof(nbytes, ms, stage):
+        return roof_hbm(nbytes, ms, peaks, traffic.get(stage))
+
+    stages = {n: tensor_roof(fl[n], st_p[n], n) for n in STAGES_P}
+    d2_ms = st_d["d2_latent_attention"]
+    stages["d2_latent_attention"] = hbm_roof(d2_own_bytes(cfgd, ctx_total, wd.batch),
+                                             d2_ms, "d2_latent_attention")
     stages["d2_latent_attention"]["tensor_executed"] = d2_tensor_view(
-        cfgd, ctx_total, st_d["d2_latent_attention"], peaks["bf16_sustained"])
+        cfgd, ctx_total, d2_ms, peaks["bf16"])
+    decode_roofline = dict(hbm_roof(dw["bytes"], dec_ms / K, "decode"),
+                           what="whole decode call (D1-D4): cache, W_kv_b, q_nope, "
+                                "q_pe and the output, over the call's event time")
     dominant = max(STAGES_P, key=lambda n: st_p[n])
     roofline = dict(stages[dominant], kernel=dominant,
-                    peak_source=f"{peaks['source']} (bf16 sustained / HBM copy)")
+                    peak_source=f"{peaks['source']} (bf16 burst / HBM copy)")
+
+    # the other prefill workloads, each timed on its own after the step
+    extra = {}
+    for name in PREFILL_OTHERS:
+        if name == args.prefill:
+            continue
+        extra[name] = time_prefill_workload(WORKLOADS[name], seeds["prefill"], K, Wm,
+                                            flush, dev, world, set_events,
+                                            tensor_roof, gpu_index(local))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -539,6 +647,8 @@ def main():
                          **{k: round(v, 4) for k, v in st_d.items()}},
             "roofline": roofline,
             "roofline_stages": stages,
+            "decode_roofline": decode_roofline,
+            "prefill_configs": extra,
             "clocks": clk,
             "gpu_launches": launches,
             "e2e": {"value": world * K * pflops / (e2e_ms * 1e-3) / 1e12,

@@ -27,9 +27,15 @@
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream).  Inputs are only read; outputs are overwritten.
  *   - Element type of activations/weights/outputs is cfg->dtype: MLA_BF16
- *     (bf16 storage, fp32 accumulation, bf16 intermediates at HBM boundaries)
- *     or MLA_F32 (fp32 throughout, CUDA-core FFMA path).  RoPE tables are
- *     always fp32; cu_ctx is int32.
+ *     (bf16 storage, fp32 accumulation, bf16 intermediates at HBM boundaries;
+ *     tensor-core kernels only) or MLA_F32 (fp32 throughout, CUDA-core FFMA
+ *     path).  RoPE tables are always fp32; cu_ctx is int32.
+ *   - MLA_BF16 shapes the tensor-core kernels take: prefill needs
+ *     qk_nope_head_dim 128, qk_rope_head_dim 64, v_head_dim 128, kv_lora_rank
+ *     a multiple of 64, hidden_size and q_lora_rank multiples of 8; decode
+ *     needs kv_lora_rank 512, qk_rope_head_dim 64, qk_nope_head_dim and
+ *     v_head_dim multiples of 8 (and hidden_size a multiple of 8 with o_proj).
+ *     Any other bf16 shape returns MLA_ERR_UNSUPPORTED before any launch.
  *   - Weights use the nn.Linear layout [out_features, in_features] and the
  *     forward computes x W^T ([MINIMIND] section 2).  There are no biases:
  *     attention_bias is False in the DeepSeek-V3 and Kimi layers ([KIMI]
@@ -410,7 +416,9 @@ MLA_API int64_t mla_kernel_launches(void);
  *   The array holds the partial slots of fewer SM pairs than a full
  *   workspace, so the decode may run on fewer SMs.  Returns MLA_ERR_WORKSPACE
  *   (with mla_last_error_detail naming both sizes) when not even one pair's
- *   layout fits, e.g. B = 16 sequences of 128 heads fit; B = 64 do not.
+ *   layout fits.  On tensor cores the scratch does not depend on max_ctx:
+ *   about 304 KiB per sequence of 128 heads plus 0.5 MiB per SM pair, so up
+ *   to B = 52 sequences of 128 heads fit (on one pair); B = 64 do not.
  *   The first call on each device looks up that device's copy of the array
  *   (cudaGetSymbolAddress) and caches it; make that first call before any
  *   stream capture.  The call allocates nothing: no cudaMalloc, cudaFree or

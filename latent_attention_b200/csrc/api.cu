@@ -227,6 +227,12 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   const int dq = dn + dr, r_kv = c.kv_lora_rank, H = c.hidden_size;
   const float eps = (float)c.rms_eps;
   const bool tc_attn = mla::tc_attention_supported(c);
+  // bf16 runs on the tensor-core kernels only
+  if (c.dtype == MLA_BF16 && (!tc_attn || H % 8 || c.q_lora_rank % 8))
+    return fail(MLA_ERR_UNSUPPORTED,
+                "bf16 prefill takes qk_nope_head_dim 128, qk_rope_head_dim 64, v_head_dim 128, "
+                "kv_lora_rank a multiple of 64, hidden_size and q_lora_rank multiples of 8 "
+                "(got %d/%d/%d, %d, %d, %d)", dn, dr, dv, r_kv, H, c.q_lora_rank);
   if (rope && (!rope_fits_simt_tiles(dq, dn, dr, h) ||
                !rope_fits_simt_tiles(r_kv + dr, r_kv, dr, 1)) && c.dtype == MLA_F32)
     return fail(MLA_ERR_UNSUPPORTED, "rope columns straddle a 64-column tile");
@@ -284,6 +290,7 @@ mla_status run_prefill(const mla_config* cfg, const mla_weights* w, const void* 
   // the column tile of the down-projection fixes the RMS partial count.
   auto run_gemm = [&](const mla::GemmArgs& ga) {
     if (mla::tc_gemm_supported(ga, c.dtype)) return mla::tc_gemm(ga, st, status);
+    if (c.dtype != MLA_F32) return cudaErrorNotSupported;   // excluded above
     if (ga.seg[0].cos && !rope_fits_simt_tiles(ga.seg[0].rope_period, ga.seg[0].rope_start,
                                                ga.seg[0].rope_dim,
                                                ga.seg[0].ncols / ga.seg[0].rope_period))
@@ -520,6 +527,13 @@ mla_status mla_decode_absorbed(const mla_config* cfg, const void* q_nope, const 
   if (!q_nope || !q_pe || !w_kv_b || !latent_cache || !cu_ctx || !out || !workspace)
     return fail(MLA_ERR_NULL, "a required decode pointer is NULL");
   if (B < 1 || B > (1 << 20) || max_ctx < 1) return fail(MLA_ERR_SHAPE, "B=%d max_ctx=%d", B, max_ctx);
+  // bf16 runs on the tensor-core kernels only
+  if (c.dtype == MLA_BF16 && (!mla::tc_decode_supported(c) || (w_o && c.hidden_size % 8)))
+    return fail(MLA_ERR_UNSUPPORTED,
+                "bf16 decode takes kv_lora_rank 512, qk_rope_head_dim 64, qk_nope_head_dim and "
+                "v_head_dim multiples of 8, hidden_size a multiple of 8 with o_proj "
+                "(got %d, %d, %d, %d, %d)", c.kv_lora_rank, c.qk_rope_head_dim,
+                c.qk_nope_head_dim, c.v_head_dim, c.hidden_size);
   const void* ptrs[] = {q_nope, q_pe, w_kv_b, latent_cache, cu_ctx, w_o, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(MLA_ERR_ALIGN, "pointer %p is not 16-byte aligned", p);

@@ -5,8 +5,8 @@
 // section 5), softmax over j, O = sum_j p_j V_h[j] with V of width v_head_dim
 // (no zero padding).  The single k_pe head is read once per key from the
 // latent buffer and shared by all heads (CSDN DeepseekV3Attention forward:
-// k_rot.expand over heads).  Used for the fp32 path and for shapes the
-// tensor-core kernel does not take.
+// k_rot.expand over heads).  The fp32 configuration's path only; bf16 runs on
+// the tensor-core attention kernel.
 #include <cfloat>
 
 #include "internal.h"
@@ -131,20 +131,12 @@ cudaError_t launch_attn_simt(int dtype, const AttnArgs& a_in, cudaStream_t st) {
   const size_t smem = sizeof(float) *
       (BQ * dq + BKEY * dq + BKEY * a.dv + BQ * BKEY + BQ * a.dv + 3 * BQ);
   dim3 grid((a.T + BQ - 1) / BQ, a.h, a.B);
-  cudaError_t err;
-  if (dtype == MLA_F32) {
-    err = cudaFuncSetAttribute(attn_simt_kernel<float>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    attn_simt_kernel<float><<<grid, NT, smem, st>>>(a);
-    count_launches();
-  } else {
-    err = cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    attn_simt_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(a);
-    count_launches();
-  }
+  if (dtype != MLA_F32) return cudaErrorNotSupported;
+  cudaError_t err = cudaFuncSetAttribute(attn_simt_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  attn_simt_kernel<float><<<grid, NT, smem, st>>>(a);
+  count_launches();
   return cudaGetLastError();
 }
 

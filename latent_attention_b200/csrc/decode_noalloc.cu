@@ -29,8 +29,14 @@ mla_status mla_decode_absorbed_noalloc(const mla_config* cfg, const void* q_nope
                                        const void* w_kv_b, const void* latent_cache,
                                        const int32_t* cu_ctx, int32_t B, int32_t max_ctx,
                                        const void* w_o, void* out, void* stream) {
-  if (!cfg) return MLA_ERR_NULL;
-  if (mla_decode_workspace_size(cfg, B, max_ctx, nullptr) == 0) return MLA_ERR_SHAPE;
+  if (!cfg) {
+    mla::set_error_detail("cfg is NULL");
+    return MLA_ERR_NULL;
+  }
+  if (mla_decode_workspace_size(cfg, B, max_ctx, nullptr) == 0) {
+    mla::set_error_detail("invalid configuration, B or max_ctx");
+    return MLA_ERR_SHAPE;
+  }
   // the array may hold fewer partial slots than the full layout: the decode
   // then runs on fewer SM pairs
   const size_t need = mla::decode_min_workspace(*cfg, B, max_ctx);
@@ -42,7 +48,15 @@ mla_status mla_decode_absorbed_noalloc(const mla_config* cfg, const void* q_nope
     return MLA_ERR_WORKSPACE;
   }
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  const cudaError_t ed = cudaGetDevice(&dev);
+  if (ed != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();   // leave no sticky runtime error behind
+    char msg[160];
+    snprintf(msg, sizeof(msg), "cudaGetDevice: %s (device %d, at most %d devices)",
+             cudaGetErrorString(ed), dev, kMaxDevices);
+    mla::set_error_detail(msg);
+    return MLA_ERR_CUDA;
+  }
   void* scratch = nullptr;
   {
     // Once per device, with that device current: the host-side name of the
@@ -50,7 +64,15 @@ mla_status mla_decode_absorbed_noalloc(const mla_config* cfg, const void* q_nope
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!g_scratch_ptr[dev]) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
+      const cudaError_t es = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (es != cudaSuccess || !p) {
+        cudaGetLastError();
+        char msg[160];
+        snprintf(msg, sizeof(msg), "cudaGetSymbolAddress of the scratch array on device %d: %s",
+                 dev, cudaGetErrorString(es));
+        mla::set_error_detail(msg);
+        return MLA_ERR_CUDA;
+      }
       g_scratch_ptr[dev] = p;
     }
     scratch = g_scratch_ptr[dev];

@@ -1,5 +1,5 @@
-// CUDA-core weight-absorbed MLA decode (fp32 math) and the latent-cache
-// finalisation used by prefill.
+// CUDA-core weight-absorbed MLA decode (the fp32 configuration) and the
+// latent-cache finalisation used by prefill (both element types).
 //
 // Megatron-LM MLA guide, 推理优化: the cache keeps [kv_compressed | k_pos_emb]
 // per token; decode folds up_k (rows [0, nope) of each head block of the kv
@@ -203,8 +203,9 @@ cudaError_t launch_latent_finalize(int dtype, const void* ckv, const float* ssq_
   return cudaGetLastError();
 }
 
+// The fp32 configuration's decode; bf16 runs on the tensor-core kernels.
 cudaError_t launch_decode_simt(int dtype, const DecodeArgs& a, cudaStream_t st) {
-  return dtype == MLA_F32 ? run_decode<float>(a, st) : run_decode<__nv_bfloat16>(a, st);
+  return dtype == MLA_F32 ? run_decode<float>(a, st) : cudaErrorNotSupported;
 }
 
 }  // namespace mla

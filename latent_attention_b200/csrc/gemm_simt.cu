@@ -1,10 +1,9 @@
 // CUDA-core GEMM with the MLA projection epilogues (fp32 FFMA).
 //
 // C = A B^T, A [M, K] row-major (stride lda), B [N, K] (nn.Linear [out, in],
-// MiniMind "Attention 前向传播" section 2).  This is the fp32 path (a tf32
-// tensor-core product cannot hold a 1e-5 relative tolerance) and the path for
-// small or odd bf16 shapes the tensor-core kernel does not take.  The
-// epilogue (see EpiSeg) fuses the RMSNorm row statistics and row scale, the
+// MiniMind "Attention 前向传播" section 2).  This is the fp32 configuration's
+// path only (a tf32 tensor-core product cannot hold a 1e-5 relative
+// tolerance); bf16 runs on the tensor-core GEMM.  The epilogue (see EpiSeg) fuses the RMSNorm row statistics and row scale, the
 // RoPE rotation of the rope columns and the RMSNorm gain.
 #include "internal.h"
 
@@ -121,11 +120,9 @@ cudaError_t launch_gemm_simt(int dtype, const GemmArgs& a, cudaStream_t st) {
   int tiles = (a.seg[0].ncols + BN - 1) / BN;
   if (a.nseg > 1) tiles += (a.seg[1].ncols + BN - 1) / BN;
   dim3 grid(tiles, (a.M + BM - 1) / BM);
+  if (dtype != MLA_F32) return cudaErrorNotSupported;
   count_launches();
-  if (dtype == MLA_F32)
-    gemm_simt_kernel<float><<<grid, NT, 0, st>>>(a);
-  else
-    gemm_simt_kernel<__nv_bfloat16><<<grid, NT, 0, st>>>(a);
+  gemm_simt_kernel<float><<<grid, NT, 0, st>>>(a);
   return cudaGetLastError();
 }
 

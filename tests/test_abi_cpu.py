@@ -231,3 +231,36 @@ def test_varlen_prefill_validation_and_sizes(lib):
     assert f(C.byref(c), C.byref(wt), p, p, 0, 10, 5, p, p, p, None, ws, big, None) == 2
     assert f(C.byref(c), C.byref(wt), p, p, 2, 10, 5, p, p, p, None, ws, C.c_size_t(64),
              None) == 5
+
+
+@pytest.mark.parametrize("field,value", [("qk_nope_head_dim", 64), ("qk_rope_head_dim", 32),
+                                         ("v_head_dim", 64), ("kv_lora_rank", 256),
+                                         ("hidden_size", 7164)])
+def test_bf16_shapes_off_the_tensor_cores_are_unsupported(lib, field, value):
+    """bf16 runs on the tensor-core kernels only: a bf16 shape they do not
+    take is refused with MLA_ERR_UNSUPPORTED before any launch (no device is
+    present here, so a launch would come back as MLA_ERR_CUDA)."""
+    from latent_attention_b200 import make_config, mla_weights
+    from latent_attention_b200._lib import mla_config
+    c = mla_config.from_buffer_copy(make_config(WORKLOADS["dsv3_prefill"].cfg))
+    setattr(c, field, value)
+    w = mla_weights()
+    for i, f in enumerate(("w_q_a", "w_q_b", "w_kv_a", "w_kv_b", "w_o")):
+        setattr(w, f, 0x100000 + i * 0x1000)
+    p, ws, big = _fake(0x200000), _fake(0x1000000), C.c_size_t(1 << 40)
+    r = lib.mla_prefill_forward(C.byref(c), C.byref(w), p, 1, 8, p, p, p, None, ws, big, None)
+    if field == "kv_lora_rank":                   # prefill takes multiples of 64
+        assert r != 6
+    else:
+        assert r == 6 and b"bf16 prefill" in lib.mla_last_error_detail()
+    dec_unsupported = field in ("qk_rope_head_dim", "kv_lora_rank")
+    # decode: kv_lora_rank 512 and rope 64; hidden_size matters with o_proj only
+    r = lib.mla_decode_absorbed(C.byref(c), p, p, p, p, p, 4, 16,
+                                p if field == "hidden_size" else None, p, ws, big, None)
+    if dec_unsupported or field == "hidden_size":
+        assert r == 6 and b"bf16 decode" in lib.mla_last_error_detail()
+    # the fp32 configuration of the same shape stays on the CUDA-core path
+    c.dtype = 0
+    if field not in ("hidden_size", "kv_lora_rank"):
+        assert lib.mla_prefill_forward(C.byref(c), C.byref(w), p, 1, 8, p, p, p, None, ws,
+                                       big, None) != 6

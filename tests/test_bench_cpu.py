@@ -31,11 +31,35 @@ def test_decode_bytes_and_executed_tensor_work():
     ctx = 1067537
     w = bench.decode_work(cfg, ctx, 64)
     assert w["cache_bytes"] == ctx * 576 * 2
+    # whole decode call: cache, W_kv_b, q_nope | q_pe in, o out
     assert w["bytes"] == ctx * 1152 + 128 * 256 * 512 * 2 + 64 * 128 * (192 + 128) * 2
+    # the latent attention kernel alone: cache, q_lat | q_pe in, o_lat out
+    # (no W_kv_b: the q-absorb and V-up GEMMs read it)
+    assert bench.d2_own_bytes(cfg, ctx, 64) == (ctx * 1152 + 64 * 128 * 576 * 2
+                                                + 64 * 128 * 512 * 2)
     v = bench.d2_tensor_view(cfg, ctx, 0.5, 1000.0)
-    # scores on both CTAs of a pair (2 x 2 x 576) plus P.C split between them
-    # (2 x 512), against the algorithmic 2 x 576 + 2 x 512 per token and head
-    assert v["flop_executed"] == ctx * 128 * 3328
+    copies = bench.D2_SCORE_COPIES
+    assert copies in (1, 2)
+    assert v["flop_executed"] == ctx * 128 * (copies * 2 * 576 + 2 * 512)
     assert v["flop_algorithmic"] == ctx * 128 * 2176
-    assert abs(v["achieved"] - ctx * 128 * 3328 / 0.5e-3 / 1e12) < 1e-9
+    assert abs(v["achieved"] - v["flop_executed"] / 0.5e-3 / 1e12) < 1e-9
     assert abs(v["frac"] - v["achieved"] / 1000.0) < 1e-12
+
+
+def test_rooflines_use_the_burst_tensor_peak_and_the_hbm_copy_rate():
+    peaks = {"bf16": 1658.8, "bf16_sustained": 1397.3, "hbm": 6550.1}
+    r = bench.roof_tensor(2.0e12, 2.0, peaks)          # 1000 TFLOP/s
+    assert r["bound"] == "tensor" and r["peak"] == 1658.8
+    assert abs(r["frac"] - 1000.0 / 1658.8) < 1e-12
+    assert abs(r["frac_sustained"] - 1000.0 / 1397.3) < 1e-12
+    h = bench.roof_hbm(3.0e9, 1.0, peaks)              # 3000 GB/s
+    assert h["bound"] == "hbm" and h["peak"] == 6550.1
+    assert abs(h["frac"] - 3000.0 / 6550.1) < 1e-12
+    assert abs(h["frac_of_8tbs"] - 3000.0 / 8000.0) < 1e-12
+
+
+def test_other_prefill_workloads_are_timed_beside_the_headline():
+    assert set(bench.PREFILL_OTHERS) == {"dsv3_prefill", "directq_prefill",
+                                         "kimi_prefill"}
+    for n in bench.PREFILL_OTHERS:
+        assert WORKLOADS[n].kind == "prefill"

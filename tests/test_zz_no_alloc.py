@@ -6,7 +6,8 @@ inputs and outputs, an allocation-free serving loop): it uses the library's
 own static device array instead of a caller workspace.  These checks call it
 through the C ABI twice in a row -- the second call reuses the array the first
 one left behind -- and compare each result with mla_decode_absorbed on the
-same inputs, at the tolerance of the other bf16 decode tests.  This file is
+same inputs and with the fp64 oracle, at the tolerance of the other bf16
+decode tests.  This file is
 collected last so that a failure here leaves every other test already run.
 """
 import pytest
@@ -26,8 +27,8 @@ TOL = 2e-2
 
 def _inputs(cfg, ctx, seed, dev, with_o):
     di = make_decode_inputs(cfg, len(ctx), ctx, seed=seed, with_o_proj=with_o)
-    return [t.to(dev) for t in (di.q_nope, di.q_pe, di.w_kv_b, di.cache,
-                                di.cu_ctx)], (di.w_o.to(dev) if with_o else None)
+    return di, [t.to(dev) for t in (di.q_nope, di.q_pe, di.w_kv_b, di.cache,
+                                    di.cu_ctx)], (di.w_o.to(dev) if with_o else None)
 
 
 @pytest.mark.parametrize("with_o", [False, True])
@@ -37,7 +38,7 @@ def test_noalloc_matches_workspace_entry_point(cuda, with_o):
     cases = [([1, 700, 4096, 65], 11), ([3000, 2, 129, 1024, 64], 12)]
     for ctx, seed in cases:                       # two calls in a row
         B = len(ctx)
-        args, w_o = _inputs(cfg, ctx, seed, cuda, with_o)
+        di, args, w_o = _inputs(cfg, ctx, seed, cuda, with_o)
         H = cfg.hidden_size if with_o else cfg.num_heads * cfg.v_head_dim
         # the full layout may exceed the array: the array's call then runs on
         # fewer SM pairs, cut at other token positions, so the two agree to
@@ -51,6 +52,11 @@ def test_noalloc_matches_workspace_entry_point(cuda, with_o):
         torch.cuda.synchronize()
         assert torch.isfinite(got.float()).all()
         assert oracle.max_rel_err(got, ref) <= TOL
+        # and both against the fp64 oracle on the same inputs
+        want = oracle.decode_absorbed(cfg, di.q_nope, di.q_pe, di.w_kv_b, di.cache,
+                                      di.cu_ctx, w_o=di.w_o if with_o else None)
+        assert oracle.max_rel_err(got, want) <= TOL
+        assert oracle.max_rel_err(ref, want) <= TOL
 
 
 def test_noalloc_rejects_oversized_requests(cuda):
