@@ -64,9 +64,10 @@ def decode_work(cfg, ctx_total, B):
             "flops": flops}
 
 
-# Score copies the latent attention kernel computes per token and head: both
-# CTAs of an SM pair compute the full scores over all r + rope dims.
-D2_SCORE_COPIES = 2
+# Score copies the latent attention kernel computes per token and head: each
+# CTA of an SM pair computes the partial scores over its own half of the
+# r + rope dims and the pair adds the two, so the scores are computed once.
+D2_SCORE_COPIES = 1
 
 
 def d2_own_bytes(cfg, ctx_total, B):

@@ -18,43 +18,46 @@
 // are cut into equal slices, one per CTA pair ("unit", one pair per two
 // SMs, a single wave), each sequence charged a fixed number of extra
 // positions for the cost of starting it (kSeqCost), so every unit has about
-// the same work whatever the length mix.  A unit walks the segments of its slice (the
-// parts of the sequences inside it) with one continuous chunk pipeline; a
-// segment covering a whole sequence writes o_lat itself, the first and last
-// segment of a slice leave a partial (o, lse) for D3.
+// the same work whatever the length mix.  A unit walks the segments of its
+// slice (the parts of the sequences inside it) with one continuous chunk
+// pipeline; a segment covering a whole sequence writes o_lat itself, the
+// first and last segment of a slice leave a partial (o, lse) for D3.
 //
 // D2 design.  With 128 heads as the MMA M dimension the latent output
 // O[128, 512] in fp32 fills all 512 TMEM columns, so the two CTAs of a unit
-// split it: CTA c accumulates latent columns [256c, 256c+256) of O (256 TMEM
-// columns).  Each CTA computes the full scores S = Q C^T over all 576 cached
-// dims itself -- the query's dims of the CTA's own latent half sit in TMEM (A
-// operand from tensor memory, 128 columns), the other half and the rope dims
-// in shared memory, so both CTAs issue the same work -- and the two CTAs need
-// no partial-score exchange and run the identical online softmax.  Each CTA
-// TMA-loads every 64-token chunk in full (9 boxes of 64 dims): the pair reads
-// the same rows at about the same time, so the second read is served by L2
-// and every cache byte crosses HBM once.  The same chunk tile is the K-major
-// B operand of S and, for the CTA's 256 latent dims, the MN-major B operand
-// of O += P C.  P_g (bf16 pairs) is written over S_g's TMEM slot.
-// A chunk's boxes form two groups with their own barriers: the 5 boxes only
-// the scores read are released as soon as the first part of S_g has run and
-// are refilled with chunk g+2 while softmax_g and PV_g are still to come; the
-// 4 value boxes of this CTA's latent columns are released by PV_g and read
-// last by S_{g+2}, so their load overlaps the first part of S_{g+2}.
+// split the latent dims: CTA c owns dims [256c, 256c + 256) and the rope
+// dims [32c, 32c + 32).  Per 64-token chunk it loads only its own four latent
+// boxes and the rope box (5 of the 9 boxes of a cache row), computes the
+// partial scores Q_c C_c^T over its own dims (the query's latent half from
+// TMEM, its rope half from shared memory) and accumulates O[:, own dims] +=
+// P C[:, own dims] from the same tiles (the K-major B operand of the scores
+// is the MN-major B operand of P C).  The two partial score tiles (128 heads
+// x 64 tokens) are exchanged through distributed shared memory as fp16 (16
+// KB each way per chunk; about 19.5 B/clk per SM of DSMEM bandwidth on B200
+// would make an fp32 exchange, 32 KB, the limit of the chunk period) and both
+// CTAs add fp16(s_0) + fp16(s_1) in fp32, the same values in the same order,
+// so the two run bit-identical online softmaxes and never exchange anything
+// else.  A group frees the chunk's TMEM score slot as soon as it has loaded
+// the partial scores, so the tensor core can compute S_{g+2} while the
+// exchange and the softmax of chunk g run; P_g (bf16) goes to shared memory
+// as the A operand of P C.
 // Between segments the query changes: the next segment's first S waits for
 // its query (both parts are reloaded once the previous segment's last S has
 // completed), and its first PV for the previous O to have been read out.  The
-// epilogue stages its TMA stores in the value boxes of the segment's last
-// chunk, which warp 2 refills only after the epilogue.
+// epilogue stages its TMA stores in the latent boxes of the segment's last
+// chunk, which the producer refills only after the epilogue.
 // Warp roles (384 threads per CTA):
-//   warp 0     TMA: each segment's query share, score-only boxes of the chunk
-//              ring (2 stages), L2 prefetch ahead (into the next segment)
+//   warp 0     TMA: the chunk ring (4 stages of 5 boxes), L2 prefetch ahead
+//              (into the next segment)
 //   warp 1     TMEM allocation, MMA issue (S_g or PV, whichever is ready)
-//   warp 2     TMA: the value boxes of the chunk ring
+//   warp 3     TMA: each segment's rope query
 //   warps 4-7, 8-11  two softmax groups taking alternate chunks (thread =
-//              head), P into TMEM; group 1 also stores each segment's TMEM
-//              query part, group 0 writes each segment's result
-// All waits are bounded; a timeout sets the device status word.
+//              head): score exchange, softmax, P into shared memory; group 1 also
+//              stores each segment's TMEM query part, group 0 writes each
+//              segment's result
+// All waits are bounded; a timeout sets the device status word.  The pair
+// passes a cluster barrier after its barriers are initialised and before it
+// exits, so no remote store or arrive reaches a CTA that is not running.
 #include <cfloat>
 
 #include "decode_slices.cuh"
@@ -70,32 +73,26 @@ using namespace slices;   // NT (tokens per chunk), the slice schedule
 constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row width
 constexpr int QBOX = 128 * 64 * 2;               // 128 heads x 64 dims bf16
 constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
-constexpr int QS_ATOMS = 5;                      // query dims [256, 576) in shared memory
-constexpr int C_ATOMS = 9;                       // a chunk's 576 dims
-constexpr int NSTAGE = 2;                        // chunk ring
+constexpr int C_BOXES = 5;                       // own latent half (4 boxes) + rope
+constexpr int NSTAGE = 4;                        // chunk ring
 constexpr int NSLOT = 2;                         // score slots
-constexpr int OFF_Q = 0;
-constexpr int OFF_C = OFF_Q + QS_ATOMS * QBOX;           // 80 KB
-constexpr int STAGE = C_ATOMS * CBOX;                    // 72 KB
+constexpr int XBUF = 128 * NT * 2;               // one chunk's fp16 partial scores, 16 KB
+constexpr int PBUF = 128 * NT * 2;               // one chunk's P (bf16), 16 KB
+constexpr int OFF_QPE = 0;                               // rope query, 16 KB
+constexpr int OFF_X = OFF_QPE + QBOX;                    // exchange buffer
+constexpr int OFF_P = OFF_X + XBUF;                      // P buffer
+constexpr int OFF_C = OFF_P + PBUF;                      // 48 KB
+constexpr int STAGE = C_BOXES * CBOX;                    // 40 KB
 constexpr int SMEM_BYTES = OFF_C + NSTAGE * STAGE + 1024;
 constexpr int NTHREADS = 384;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
-// TMEM: score slots [0, 128) (64 columns each; P_j over the first 32 of slot
-// j % 2), O [128, 384), the query's latent dims [256c, 256c + 256) of CTA c
-// as bf16 pairs [384, 512).
+// TMEM: score slots [0, 128) (64 columns each), O [128, 384), the query's
+// latent dims [256c, 256c + 256) of CTA c as bf16 pairs [384, 512).
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_Q = 384;
 constexpr float kRescaleLog2 = 8.f;
-constexpr int SO_BOXES = 5, V_BOXES = 4;      // score-only / value boxes of a chunk
 constexpr int EPI_BOX = 32 * 128;             // epilogue staging: 32 rows of 128 bytes
-
-// Box i of the score-only group of the CTA with cluster rank `rank` (the
-// latent half the CTA does not accumulate, then the rope box); the value
-// group of rank c is boxes 4c .. 4c + 3.
-__device__ __forceinline__ int score_only_box(uint32_t rank, int i) {
-  return i < 4 ? (rank ? i : 4 + i) : 8;
-}
 
 struct DecTcParams {
   const int32_t* cu_ctx;
@@ -108,6 +105,26 @@ struct DecTcParams {
   __nv_bfloat16* o_lat;        // [B, h, R]
   uint32_t* status;
 };
+
+// Bounded wait until a shared counter reaches `target` (same limit and abort
+// protocol as the barrier waits).
+__device__ __forceinline__ bool wait_count(const int* counter, int target,
+                                           volatile int* abort_flag, uint32_t* status) {
+  const volatile int* c = counter;
+  if (*c >= target) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (*c >= target) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitNs) {
+        *abort_flag = 1;
+        if (status) atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
 
 // First token (relative to the sequence start) of the 64-row box that chunk j
 // of a split starting at token t0 loads.  A box never reaches past the last
@@ -129,9 +146,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                        const __grid_constant__ CUtensorMap tmOL,
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, qt_full, q_free, ca_full[NSTAGE], ca_empty[NSTAGE],
-      cb_full[NSTAGE], cb_empty[NSTAGE], s_full[NSLOT], p_full[NSLOT], pv_done[2], o_done,
-      o_free, ref_ready[2];
+  __shared__ __align__(8) uint64_t q_full, qt_full, q_free, c_full[NSTAGE], c_empty[NSTAGE],
+      s_full[NSLOT], s_free[NSLOT], x_full[2], x_empty[2], p_full, pv_done[2], o_done, o_free,
+      ref_ready[2];
+  __shared__ int epi_count;                    // epilogue warps done, all segments
   __shared__ float m_hand[128];                // reference max after the last chunk
   __shared__ float fin_m[128], fin_l[128];      // group 1's state at a segment's end
   __shared__ uint32_t tmem_base;
@@ -147,7 +165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int32_t* cu = p.cu_ctx;
   const Slice sl = unit_slice(cu, p.B, p.max_ctx, u, p.n_units, p.min_len);
   if (sl.r0 >= sl.r1) return;                    // past the end of the stream (both CTAs)
-  const int dim0 = 256 * (int)rank;              // this CTA's latent columns of O
+  const int dim0 = 256 * (int)rank;              // this CTA's latent columns
 
   if (threadIdx.x == 0) {
     seq_lo = seq_at(cu, p.B, sl.r0);
@@ -156,17 +174,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     mbar_init(&qt_full, 4);         // softmax group 1 stored the TMEM query part
     mbar_init(&q_free, 1);          // the last S of a segment completed
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&ca_full[s], 1);
-      mbar_init(&ca_empty[s], 1);
-      mbar_init(&cb_full[s], 1);
-      mbar_init(&cb_empty[s], 1);
+      mbar_init(&c_full[s], 1);
+      mbar_init(&c_empty[s], 1);
     }
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);     // the chunk's softmax group wrote P_g
+      mbar_init(&s_free[s], 4);     // the chunk's softmax group loaded S_g
     }
-    mbar_init(&pv_done[0], 1);
-    mbar_init(&pv_done[1], 1);
+    // The exchange buffer and the P buffer hold one chunk at a time, but
+    // their barriers come in pairs by chunk parity (phase g >> 1 of barrier
+    // g & 1), so that no waiter ever looks for a phase two ahead of the
+    // current one (a parity wait would take the older phase for it).
+    // x_full[x] counts the bytes of the peer's partial scores of a chunk
+    // (armed for chunks 0 and 1 here, then for chunk g + 2 by the group that
+    // has seen chunk g arrive); x_empty[x] completes when the peer's group has
+    // read this CTA's partial scores; pv_done[x] when PV_g has run.  p_full
+    // (P_g written) is waited for in chunk order by the MMA warp alone.
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&x_full[x], 1);
+      mbar_arrive_expect_tx(&x_full[x], XBUF);
+      mbar_init(&x_empty[x], 4);
+      mbar_init(&pv_done[x], 1);
+    }
+    mbar_init(&p_full, 4);
+    epi_count = 0;
     mbar_init(&o_done, 1);          // the last PV of a segment completed
     mbar_init(&o_free, 4);          // softmax group 0 has read O out of TMEM
     mbar_init(&ref_ready[0], 4);    // a softmax group published chunk g's reference
@@ -179,6 +210,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
   }
   __syncthreads();
+  cluster_sync_all();               // the peer's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tbase = tmem_base;
   const int b0 = seq_lo, b1 = seq_hi;
@@ -186,23 +218,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int sm_wg = (warp >= 4 && warp < 8) ? 0 : (warp >= 8 ? 1 : -1);
 
   if (warp == 0) {
-    // ---------------- query share of each segment, score-only boxes, L2 prefetch
+    // ---------------- the chunk ring, L2 prefetch
     if (elect_one()) {
       tma_prefetch(&tmQ);
-      tma_prefetch(&tmQpe);
       tma_prefetch(&tmC);
+      // this CTA's boxes of chunk j of segment s into L2 (the rope box by rank 0)
       auto prefetch = [&](const Seg& s, int j) {
-        for (int a = 0; a < C_ATOMS; ++a)
-          tma_prefetch_l2_2d(&tmC, 64 * a, (int)s.start + chunk_base(s.n, s.t0, j));
+        const int y = (int)s.start + chunk_base(s.n, s.t0, j);
+        for (int a = 0; a < 4; ++a) tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, y);
+        if (rank == 0) tma_prefetch_l2_2d(&tmC, R, y);
       };
-      // the query rows of a segment (all 576 dims) into L2
+      // this CTA's latent half of a segment's query rows into L2
       auto prefetch_q = [&](const Seg& s) {
-        for (int a = 0; a < 8; ++a) tma_prefetch_l2_2d(&tmQ, 64 * a, s.b * p.h + h0);
-        tma_prefetch_l2_2d(&tmQpe, 0, s.b * p.h + h0);
+        for (int a = 0; a < 4; ++a) tma_prefetch_l2_2d(&tmQ, dim0 + 64 * a, s.b * p.h + h0);
       };
       SegCursor c, nx;
       c.start(cu, b0, b1, p.max_ctx, sl, u);
       int prev_nch = 0;
+      // a stage whose last chunk ended a segment also holds that segment's
+      // epilogue staging: segment ordinal, or -1
+      int staged[NSTAGE];
+      for (int s = 0; s < NSTAGE; ++s) staged[s] = -1;
       for (int g = 0; !c.done; ++g) {
         const Seg& s = c.s;
         if (c.j == 0) {
@@ -211,13 +247,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           prev_nch = s.nch;
           nx = c;                          // the next segment, prefetched near this one's end
           nx.next_seg(cu, b0, b1, p.max_ctx, sl, u);
-          // the previous segment's scores no longer read the query buffer
-          if (c.kk > 0 && !mbar_wait(&q_free, (c.kk - 1) & 1, abort_v, p.status)) break;
-          mbar_arrive_expect_tx(&q_full, QS_ATOMS * QBOX);
-          for (int a = 0; a < 4; ++a)      // the other CTA's latent half of the query
-            tma_load_2d(smem + OFF_Q + a * QBOX, &tmQ, (256 - dim0) + 64 * a, s.b * p.h + h0,
-                        &q_full);
-          tma_load_2d(smem + OFF_Q + 4 * QBOX, &tmQpe, 0, s.b * p.h + h0, &q_full);
         }
         if (c.j + PREFETCH < s.nch) {
           prefetch(s, c.j + PREFETCH);
@@ -227,115 +256,93 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           if (jn < nx.s.nch) prefetch(nx.s, jn);
         }
         const int st = g % NSTAGE;
-        if (!mbar_wait(&ca_empty[st], ((g / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+        if (!mbar_wait(&c_empty[st], ((g / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
+        // (a count, not a barrier phase: this wait may lag several segments)
+        if (staged[st] >= 0 &&
+            !wait_count(&epi_count, 4 * (staged[st] + 1), abort_v, p.status))
+          break;
+        staged[st] = c.j == s.nch - 1 ? c.kk : -1;
         uint8_t* sc = smem + OFF_C + st * STAGE;
-        mbar_arrive_expect_tx(&ca_full[st], SO_BOXES * CBOX);
+        mbar_arrive_expect_tx(&c_full[st], C_BOXES * CBOX);
         const int y = (int)s.start + chunk_base(s.n, s.t0, c.j);
-        for (int i = 0; i < SO_BOXES; ++i) {
-          const int a = score_only_box(rank, i);
-          tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &ca_full[st]);
-        }
+        for (int a = 0; a < 4; ++a) tma_load_2d(sc + a * CBOX, &tmC, dim0 + 64 * a, y, &c_full[st]);
+        tma_load_2d(sc + 4 * CBOX, &tmC, R, y, &c_full[st]);
         c.next(cu, b0, b1, p.max_ctx, sl, u);
       }
     }
-  } else if (warp == 2) {
-    // ---------------- value boxes
+  } else if (warp == 3) {
+    // ---------------- each segment's rope query (shared memory A operand)
     if (elect_one()) {
+      tma_prefetch(&tmQpe);
       SegCursor c;
       c.start(cu, b0, b1, p.max_ctx, sl, u);
-      // a stage whose last chunk ended a segment also holds that segment's
-      // epilogue staging: segment ordinal, or -1
-      int staged[NSTAGE] = {-1, -1};
-      for (int g = 0; !c.done; ++g) {
-        const Seg& s = c.s;
-        const int st = g % NSTAGE;
-        if (!mbar_wait(&cb_empty[st], ((g / NSTAGE) & 1) ^ 1, abort_v, p.status)) break;
-        if (staged[st] >= 0 && !mbar_wait(&o_free, staged[st] & 1, abort_v, p.status)) break;
-        staged[st] = c.j == s.nch - 1 ? c.kk : -1;
-        uint8_t* sc = smem + OFF_C + st * STAGE;
-        mbar_arrive_expect_tx(&cb_full[st], V_BOXES * CBOX);
-        const int y = (int)s.start + chunk_base(s.n, s.t0, c.j);
-        for (int i = 0; i < V_BOXES; ++i) {
-          const int a = 4 * (int)rank + i;
-          tma_load_2d(sc + a * CBOX, &tmC, 64 * a, y, &cb_full[st]);
-        }
-        c.next(cu, b0, b1, p.max_ctx, sl, u);
+      for (; !c.done; c.next_seg(cu, b0, b1, p.max_ctx, sl, u)) {
+        // the previous segment's scores no longer read the buffer
+        if (c.kk > 0 && !mbar_wait(&q_free, (c.kk - 1) & 1, abort_v, p.status)) break;
+        mbar_arrive_expect_tx(&q_full, QBOX);
+        tma_load_2d(smem + OFF_QPE, &tmQpe, 0, c.s.b * p.h + h0, &q_full);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issue
     if (elect_one()) {
-      const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_Q));
-      // S_g += Q box a . C_g box a^T (four MMAs of 16 dims): query dims
-      // [0, 256) from TMEM, the rest from shared memory; dc describes the
-      // chunk's stage
-      auto s_box = [&](uint32_t d, uint64_t dc, int a, bool first) {
-        if (a < 8 && (a >> 2) == (int)rank) {   // this CTA's latent half: query in TMEM
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ts(d, tbase + TM_Q + (a & 3) * 32 + k * 8,
-                        dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
-        } else {                                 // the other half and rope: shared memory
-          const int qa = a < 8 ? (a & 3) : 4;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(d, dq + (uint64_t)((qa * QBOX + k * 32) >> 4),
-                     dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, !(first && k == 0));
-        }
-      };
+      const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_QPE));
       // Issue S_gs and O += P_gp C_gp in whichever order their inputs become
-      // ready, across segments.  S_gs reuses the slot of S/P_{gs-2}, so it
-      // follows PV_{gs-2} in issue order (gs < gp + 2), which is execution
-      // order; PV_gp follows S_gp.  S_gs goes out in two parts: the
-      // score-only boxes, then the value boxes.  A segment's first S waits
-      // for its query (shared memory and TMEM parts), its first PV for the
-      // previous segment's O to have been read out.
+      // ready, across segments.  S_gs reuses the slot of S_{gs-2} once that
+      // chunk's softmax group has loaded it; PV_gp follows S_gp.  A
+      // segment's first S waits for its query (shared memory and TMEM
+      // parts), its first PV for the previous segment's O to have been read
+      // out.
       SegCursor cs, cp;
       cs.start(cu, b0, b1, p.max_ctx, sl, u);
       cp.start(cu, b0, b1, p.max_ctx, sl, u);
       int gs = 0, gp = 0;
-      bool s_part = false, ok = true;      // s_part: S_gs's score-only part is issued
+      bool ok = true;
       uint64_t t_stall = 0;
       uint32_t idle = 0;
       while (ok && !cp.done) {
         bool progress = false;
-        if (!cs.done && gs < gp + NSLOT) {
+        if (!cs.done) {
           const int st = gs % NSTAGE, sls = gs % NSLOT;
-          const uint32_t par = (gs / NSTAGE) & 1;
           const uint32_t d = tbase + TM_S + sls * NT;
           const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
-          if (!s_part &&
-              (cs.j != 0 || (mbar_test(&q_full, cs.kk & 1) && mbar_test(&qt_full, cs.kk & 1))) &&
-              mbar_test(&ca_full[st], par)) {
+          if ((cs.j != 0 || (mbar_test(&q_full, cs.kk & 1) && mbar_test(&qt_full, cs.kk & 1))) &&
+              (gs < NSLOT || mbar_test(&s_free[sls], ((gs / NSLOT) - 1) & 1)) &&
+              mbar_test(&c_full[st], (gs / NSTAGE) & 1)) {
             tc_fence_after();
-            for (int i = 0; i < SO_BOXES; ++i) s_box(d, dc, score_only_box(rank, i), i == 0);
-            mma_commit(&ca_empty[st]);
-            s_part = true;
-            progress = true;
-          }
-          if (s_part && mbar_test(&cb_full[st], par)) {
-            tc_fence_after();
-            for (int i = 0; i < V_BOXES; ++i) s_box(d, dc, 4 * (int)rank + i, false);
+            // partial S_gs over this CTA's dims: its latent half (query in
+            // TMEM) and its half of the rope dims (query in shared memory)
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts(d, tbase + TM_Q + a * 32 + k * 8,
+                            dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, (a | k) != 0);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int kr = 2 * (int)rank + k;
+              mma_bf16(d, dq + (uint64_t)((kr * 32) >> 4),
+                       dc + (uint64_t)((4 * CBOX + kr * 32) >> 4), IDESC_S, 1);
+            }
             mma_commit(&s_full[sls]);
             if (cs.j == cs.s.nch - 1) mma_commit(&q_free);
-            s_part = false;
             ++gs;
             cs.next(cu, b0, b1, p.max_ctx, sl, u);
             progress = true;
           }
         }
         if (gp < gs) {
-          const int st = gp % NSTAGE, slp = gp % NSLOT;
-          if (mbar_test(&p_full[slp], (gp / NSLOT) & 1) &&
+          const int st = gp % NSTAGE;
+          if (mbar_test(&p_full, gp & 1) &&
               (cp.j != 0 || cp.kk == 0 || mbar_test(&o_free, (cp.kk - 1) & 1))) {
             tc_fence_after();
-            const uint64_t dv =
-                desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE + (dim0 / 64) * CBOX), CBOX);
+            const uint64_t dv = desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE), CBOX);
+            const uint64_t dp = desc_kmajor_sw128(smem_u32(smem + OFF_P));
 #pragma unroll
             for (int k = 0; k < NT / 16; ++k)
-              mma_bf16_ts(tbase + TM_O, tbase + TM_S + slp * NT + k * 8,
-                          dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (cp.j | k) != 0);
-            mma_commit(&cb_empty[st]);
+              mma_bf16(tbase + TM_O, dp + (uint64_t)((k * 32) >> 4),
+                       dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (cp.j | k) != 0);
+            mma_commit(&c_empty[st]);
             mma_commit(&pv_done[gp & 1]);
             if (cp.j == cp.s.nch - 1) mma_commit(&o_done);
             ++gp;
@@ -360,16 +367,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
   } else if (sm_wg >= 0) {
     // ---------------- softmax (thread = head): group g takes the chunks of
-    // its parity in the unit's chunk sequence (score slot g).  The reference
-    // max of every row passes from one group to the other through shared
-    // memory; each group keeps the row sum of its own chunks, relative to its
-    // last reference.  Per segment, group 1 first stores the query's TMEM
-    // part, group 0 finally merges both groups' sums and writes the result.
+    // its parity in the unit's chunk sequence (score slot and exchange
+    // buffer g).  The reference max of every row passes from one group to the
+    // other through shared memory; each group keeps the row sum of its own
+    // chunks, relative to its last reference.  Per segment, group 1 first
+    // stores the query's TMEM part, group 0 finally merges both groups' sums
+    // and writes the result.
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int head = h0 + r;
     const bool head_ok = head < p.h;
+    // this head's 16-byte column of the exchange buffer (16-byte piece k of
+    // row r at k * 2048 + 16 r, so a warp's stores are 512 contiguous bytes),
+    // here and in the peer; its 128-byte row of the P buffer (the 128-byte
+    // swizzled K-major layout of an MMA operand)
+    const uint32_t x_mine = smem_u32(smem + OFF_X) + r * 16;
+    const uint32_t x_peer = mapa_shared(x_mine, rank ^ 1u);
+    const uint32_t p_row = smem_u32(smem + OFF_P) + r * 128;
+    // the peer's x_full / x_empty barriers (those of parity x 8 bytes further)
+    const uint32_t peer_x_full = mapa_shared(smem_u32(&x_full[0]), rank ^ 1u);
+    const uint32_t peer_x_empty = mapa_shared(smem_u32(&x_empty[0]), rank ^ 1u);
     bool ok = true;
     SegCursor c;
     c.start(cu, b0, b1, p.max_ctx, sl, u);
@@ -416,16 +434,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (int j = 0; ok && j < s.nch; ++j) {
         const int g = g0 + j;
         if ((g & 1) != sm_wg) continue;
-        const int sls = g % NSLOT, xs = g & 1;
+        const int sls = g % NSLOT, xs = g & 1;   // score slot; the group's hand-over slot
         if (!warp_wait(&s_full[sls], (g / NSLOT) & 1, abort_v, p.status)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[2][32];
-        tmem_ld32(tbase + lane_off + TM_S + sls * NT, sr[0]);
-        tmem_ld32(tbase + lane_off + TM_S + sls * NT + 32, sr[1]);
-        tmem_wait_ld();
+        // this CTA's partial scores as fp16 pairs
+        uint32_t hx[32];
+        {
+          uint32_t sr[2][32];
+          tmem_ld32(tbase + lane_off + TM_S + sls * NT, sr[0]);
+          tmem_ld32(tbase + lane_off + TM_S + sls * NT + 32, sr[1]);
+          tmem_wait_ld();
+          tc_fence_before();      // the slot may take S_{g+2}
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[sls]);
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            hx[e] = pack_f16_sat(__uint_as_float(sr[e >> 4][(2 * e) & 31]),
+                                 __uint_as_float(sr[e >> 4][(2 * e + 1) & 31]));
+        }
+        // into the peer's exchange buffer, once the peer has read chunk g - 1
+        // there: asynchronous stores that count their bytes on its x_full
+        if (g >= 1 &&
+            !warp_wait(&x_empty[xs ^ 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_async_v4(x_peer + k * 2048, peer_x_full + 8 * xs, hx[4 * k], hx[4 * k + 1],
+                      hx[4 * k + 2], hx[4 * k + 3]);
+        // the peer's partial scores of chunk g; then x_full[xs] is armed for
+        // chunk g + 2, whose bytes the peer sends only after chunk g + 1 has
+        // been read here, which follows this group's reading of chunk g
+        if (!warp_wait_cluster(&x_full[xs], (g >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        if (quad == 0 && lane == 0) mbar_arrive_expect_tx(&x_full[xs], XBUF);
         float sv[NT];
 #pragma unroll
-        for (int i = 0; i < NT; ++i) sv[i] = __uint_as_float(sr[i >> 5][i & 31]);
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = ld_shared_v4(x_mine + k * 2048);
+          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float a0, a1, b0, b1;
+            unpack_f16(hx[4 * k + i], a0, a1);
+            unpack_f16(pv[i], b0, b1);
+            sv[8 * k + 2 * i] = a0 + b0;          // the same sum on both CTAs
+            sv[8 * k + 2 * i + 1] = a1 + b1;
+          }
+        }
+        __syncwarp();   // the values are summed: the buffer may take chunk g + 1
+        if (lane == 0) mbar_arrive_cluster_relaxed(peer_x_empty + 8 * xs);
         // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
         const int base = chunk_base(s.n, s.t0, j) - s.t0;
         const int lo = j * NT - base, hi = s.tcount - base;
@@ -476,15 +537,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           w[e] = pack_bf16(p0, p1);
         }
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        // O holds the segment's sum through chunk j-1 at reference m_prev:
-        // rescale it when this chunk moved the reference (PV_{g-1} must be
-        // complete).
+        // PV_{g-1} has run: it no longer reads the P buffer, and O holds the
+        // segment's sum through chunk j-1 at reference m_prev -- rescale it
+        // when this chunk moved the reference.
+        if (g >= 1 &&
+            !warp_wait(&pv_done[xs ^ 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
           const float alpha = ex2(m_prev - m_new);
-          if (!warp_wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < 8; ++cc) {
@@ -495,13 +557,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(tbase + lane_off + TM_O + cc * 32, o);
           }
+          tmem_wait_st();
         }
-        // P_g over the first half of S_g's slot (S_g is in registers already)
-        tmem_st32(tbase + lane_off + TM_S + sls * NT, w);
-        tmem_wait_st();
-        tc_fence_before();
+        // P_g into the P buffer
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(p_row + ((k ^ (r & 7)) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
+                       w[4 * k + 3]);
+        fence_proxy_async();
+        tc_fence_before();        // the O rescale above happens before PV_g
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sls]);
+        if (lane == 0) mbar_arrive(&p_full);
       }
       g0 += s.nch;
       // Segment end.  Both groups' sums at the last chunk's reference
@@ -524,16 +590,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                               (l1 > 0.f ? l1 * ex2(m1 - m_last) : 0.f);
           const float inv = 1.f / l_tot;
           tc_fence_after();
-          // This warp's 32 rows go out through the value boxes of the
-          // segment's last chunk (free: its PV has completed; warp 2 refills
+          // This warp's 32 rows go out through the latent boxes of the
+          // segment's last chunk (free: its PV has completed; warp 0 refills
           // them only after o_free) and TMA stores, 32 x 64 bf16 or
           // 32 x 32 fp32 per box; a warp whose rows straddle the head count
           // stores directly.
           const int row0 = h0 + quad * 32;
           const bool tma_rows = row0 + 32 <= p.h;
           const int g_last = g0 - 1;
-          const uint32_t stg = smem_u32(smem + OFF_C + (g_last % NSTAGE) * STAGE) +
-                               4 * rank * CBOX + quad * 2 * EPI_BOX;
+          const uint32_t stg =
+              smem_u32(smem + OFF_C + (g_last % NSTAGE) * STAGE) + quad * 2 * EPI_BOX;
           auto stage = [&](int i, const uint32_t (&v)[32]) -> uint32_t {
             const uint32_t sb = stg + (i & 1) * EPI_BOX;
             if (i >= 2) {             // the store issued from this box two boxes ago
@@ -600,8 +666,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (rank == 0 && head_ok)
               p.part_lse[part] = (m_last + __log2f(l_tot)) * 0.6931471805599453f;
           }
-          // the staging boxes are read out before warp 2 refills them
-          if (lane == 0) bulk_wait_group_read<0>();
+          // the staging boxes are read out before warp 0 refills them
+          if (lane == 0) {
+            bulk_wait_group_read<0>();
+            atomicAdd(&epi_count, 1);
+          }
           __syncwarp();
           // O may be overwritten by the next segment's first PV
           tc_fence_before();
@@ -615,6 +684,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  // both CTAs are done with each other's shared memory
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
