@@ -26,12 +26,12 @@
 // D2 design.  With 128 heads as the MMA M dimension the latent output
 // O[128, 512] in fp32 fills all 512 TMEM columns, so the two CTAs of a unit
 // split the latent dims: CTA c owns dims [256c, 256c + 256) and the rope
-// dims [32c, 32c + 32).  Per 64-token chunk it loads only its own four latent
-// boxes and the rope box (5 of the 9 boxes of a cache row), computes the
-// partial scores Q_c C_c^T over its own dims (the query's latent half from
-// TMEM, its rope half from shared memory) and accumulates O[:, own dims] +=
-// P C[:, own dims] from the same tiles (the K-major B operand of the scores
-// is the MN-major B operand of P C).  The two partial score tiles (128 heads
+// dims [32c, 32c + 32).  Per 64-token chunk it loads only its own half of
+// every cache row (four 64-dim latent boxes and a 32-dim rope box with
+// 64-byte swizzle, 36 KB), computes the partial scores Q_c C_c^T over its own
+// dims (the query's latent half from TMEM, its rope half from shared memory)
+// and accumulates O[:, own dims] += P C[:, own dims] from the same tiles (the
+// K-major B operand of the scores is the MN-major B operand of P C).  The two partial score tiles (128 heads
 // x 64 tokens) are exchanged through distributed shared memory as fp16 (16
 // KB each way per chunk; about 19.5 B/clk per SM of DSMEM bandwidth on B200
 // would make an fp32 exchange, 32 KB, the limit of the chunk period) and both
@@ -47,10 +47,10 @@
 // epilogue stages its TMA stores in the latent boxes of the segment's last
 // chunk, which the producer refills only after the epilogue.
 // Warp roles (384 threads per CTA):
-//   warp 0     TMA: the chunk ring (4 stages of 5 boxes), L2 prefetch ahead
+//   warp 0     TMA: the chunk ring (5 stages of 36 KB), L2 prefetch ahead
 //              (into the next segment)
 //   warp 1     TMEM allocation, MMA issue (S_g or PV, whichever is ready)
-//   warp 3     TMA: each segment's rope query
+//   warp 3     TMA: each segment's rope query (this CTA's half)
 //   warps 4-7, 8-11  two softmax groups taking alternate chunks (thread =
 //              head): score exchange, softmax, P into shared memory; group 1 also
 //              stores each segment's TMEM query part, group 0 writes each
@@ -71,18 +71,18 @@ using namespace sm100;
 using namespace slices;   // NT (tokens per chunk), the slice schedule
 
 constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row width
-constexpr int QBOX = 128 * 64 * 2;               // 128 heads x 64 dims bf16
+constexpr int QPE_BOX = 128 * 32 * 2;            // 128 heads x this CTA's 32 rope dims
 constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
-constexpr int C_BOXES = 5;                       // own latent half (4 boxes) + rope
-constexpr int NSTAGE = 4;                        // chunk ring
+constexpr int RBOX = NT * 32 * 2;                // 64 tokens x this CTA's 32 rope dims
+constexpr int NSTAGE = 5;                        // chunk ring
 constexpr int NSLOT = 2;                         // score slots
 constexpr int XBUF = 128 * NT * 2;               // one chunk's fp16 partial scores, 16 KB
 constexpr int PBUF = 128 * NT * 2;               // one chunk's P (bf16), 16 KB
-constexpr int OFF_QPE = 0;                               // rope query, 16 KB
-constexpr int OFF_X = OFF_QPE + QBOX;                    // exchange buffer
+constexpr int OFF_QPE = 0;                               // rope query half, 8 KB
+constexpr int OFF_X = OFF_QPE + QPE_BOX;                 // exchange buffer
 constexpr int OFF_P = OFF_X + XBUF;                      // P buffer
-constexpr int OFF_C = OFF_P + PBUF;                      // 48 KB
-constexpr int STAGE = C_BOXES * CBOX;                    // 40 KB
+constexpr int OFF_C = OFF_P + PBUF;                      // 40 KB
+constexpr int STAGE = 4 * CBOX + RBOX;                   // 36 KB
 constexpr int SMEM_BYTES = OFF_C + NSTAGE * STAGE + 1024;
 constexpr int NTHREADS = 384;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
@@ -142,6 +142,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmQpe,
                        const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmCr,
                        const __grid_constant__ CUtensorMap tmPO,
                        const __grid_constant__ CUtensorMap tmOL,
                        const __grid_constant__ DecTcParams p) {
@@ -222,11 +223,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (elect_one()) {
       tma_prefetch(&tmQ);
       tma_prefetch(&tmC);
-      // this CTA's boxes of chunk j of segment s into L2 (the rope box by rank 0)
+      tma_prefetch(&tmCr);
+      // this CTA's boxes of chunk j of segment s into L2
       auto prefetch = [&](const Seg& s, int j) {
         const int y = (int)s.start + chunk_base(s.n, s.t0, j);
         for (int a = 0; a < 4; ++a) tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, y);
-        if (rank == 0) tma_prefetch_l2_2d(&tmC, R, y);
+        tma_prefetch_l2_2d(&tmCr, R + 32 * (int)rank, y);
       };
       // this CTA's latent half of a segment's query rows into L2
       auto prefetch_q = [&](const Seg& s) {
@@ -263,10 +265,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           break;
         staged[st] = c.j == s.nch - 1 ? c.kk : -1;
         uint8_t* sc = smem + OFF_C + st * STAGE;
-        mbar_arrive_expect_tx(&c_full[st], C_BOXES * CBOX);
+        mbar_arrive_expect_tx(&c_full[st], STAGE);
         const int y = (int)s.start + chunk_base(s.n, s.t0, c.j);
         for (int a = 0; a < 4; ++a) tma_load_2d(sc + a * CBOX, &tmC, dim0 + 64 * a, y, &c_full[st]);
-        tma_load_2d(sc + 4 * CBOX, &tmC, R, y, &c_full[st]);
+        tma_load_2d(sc + 4 * CBOX, &tmCr, R + 32 * (int)rank, y, &c_full[st]);
         c.next(cu, b0, b1, p.max_ctx, sl, u);
       }
     }
@@ -279,14 +281,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (; !c.done; c.next_seg(cu, b0, b1, p.max_ctx, sl, u)) {
         // the previous segment's scores no longer read the buffer
         if (c.kk > 0 && !mbar_wait(&q_free, (c.kk - 1) & 1, abort_v, p.status)) break;
-        mbar_arrive_expect_tx(&q_full, QBOX);
-        tma_load_2d(smem + OFF_QPE, &tmQpe, 0, c.s.b * p.h + h0, &q_full);
+        mbar_arrive_expect_tx(&q_full, QPE_BOX);
+        tma_load_2d(smem + OFF_QPE, &tmQpe, 32 * (int)rank, c.s.b * p.h + h0, &q_full);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issue
     if (elect_one()) {
-      const uint64_t dq = desc_kmajor_sw128(smem_u32(smem + OFF_QPE));
+      const uint64_t dq = desc_kmajor_sw64(smem_u32(smem + OFF_QPE));
       // Issue S_gs and O += P_gp C_gp in whichever order their inputs become
       // ready, across segments.  S_gs reuses the slot of S_{gs-2} once that
       // chunk's softmax group has loaded it; PV_gp follows S_gp.  A
@@ -302,35 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       uint32_t idle = 0;
       while (ok && !cp.done) {
         bool progress = false;
-        if (!cs.done) {
-          const int st = gs % NSTAGE, sls = gs % NSLOT;
-          const uint32_t d = tbase + TM_S + sls * NT;
-          const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
-          if ((cs.j != 0 || (mbar_test(&q_full, cs.kk & 1) && mbar_test(&qt_full, cs.kk & 1))) &&
-              (gs < NSLOT || mbar_test(&s_free[sls], ((gs / NSLOT) - 1) & 1)) &&
-              mbar_test(&c_full[st], (gs / NSTAGE) & 1)) {
-            tc_fence_after();
-            // partial S_gs over this CTA's dims: its latent half (query in
-            // TMEM) and its half of the rope dims (query in shared memory)
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts(d, tbase + TM_Q + a * 32 + k * 8,
-                            dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, (a | k) != 0);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int kr = 2 * (int)rank + k;
-              mma_bf16(d, dq + (uint64_t)((kr * 32) >> 4),
-                       dc + (uint64_t)((4 * CBOX + kr * 32) >> 4), IDESC_S, 1);
-            }
-            mma_commit(&s_full[sls]);
-            if (cs.j == cs.s.nch - 1) mma_commit(&q_free);
-            ++gs;
-            cs.next(cu, b0, b1, p.max_ctx, sl, u);
-            progress = true;
-          }
-        }
+        // PV first: its completion frees the chunk's stage
         if (gp < gs) {
           const int st = gp % NSTAGE;
           if (mbar_test(&p_full, gp & 1) &&
@@ -347,6 +321,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (cp.j == cp.s.nch - 1) mma_commit(&o_done);
             ++gp;
             cp.next(cu, b0, b1, p.max_ctx, sl, u);
+            progress = true;
+          }
+        }
+        if (!cs.done) {
+          const int st = gs % NSTAGE, sls = gs % NSLOT;
+          const uint32_t d = tbase + TM_S + sls * NT;
+          const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
+          if ((cs.j != 0 || (mbar_test(&q_full, cs.kk & 1) && mbar_test(&qt_full, cs.kk & 1))) &&
+              (gs < NSLOT || mbar_test(&s_free[sls], ((gs / NSLOT) - 1) & 1)) &&
+              mbar_test(&c_full[st], (gs / NSTAGE) & 1)) {
+            tc_fence_after();
+            // partial S_gs over this CTA's dims: its latent half (query in
+            // TMEM) and its half of the rope dims (query in shared memory)
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts(d, tbase + TM_Q + a * 32 + k * 8,
+                            dc + (uint64_t)((a * CBOX + k * 32) >> 4), IDESC_S, (a | k) != 0);
+            const uint64_t dr = desc_kmajor_sw64(smem_u32(smem + OFF_C + st * STAGE + 4 * CBOX));
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+              mma_bf16(d, dq + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), IDESC_S, 1);
+            mma_commit(&s_full[sls]);
+            if (cs.j == cs.s.nch - 1) mma_commit(&q_free);
+            ++gs;
+            cs.next(cu, b0, b1, p.max_ctx, sl, u);
             progress = true;
           }
         }
@@ -774,20 +775,22 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
   stage_event(1, st);
   // D2
   {
-    CUtensorMap tmQ, tmQpe, tmC;
+    CUtensorMap tmQ, tmQpe, tmC, tmCr;
     const uint32_t qbox[2] = {64, 128}, cbox[2] = {64, NT};
+    const uint32_t qpebox[2] = {32, 128}, rbox[2] = {32, NT};   // a CTA's rope half
     const uint64_t qdims[2] = {(uint64_t)R, (uint64_t)a.B * a.h};
     const uint64_t qstr[1] = {(uint64_t)R * 2};
     if (!encode_tmap(&tmQ, a.q_lat, 2, qdims, qstr, qbox)) return cudaErrorInvalidValue;
     const uint64_t pdims[2] = {(uint64_t)DR, (uint64_t)a.B * a.h};
     const uint64_t pstr[1] = {(uint64_t)DR * 2};
-    if (!encode_tmap(&tmQpe, a.q_pe, 2, pdims, pstr, qbox)) return cudaErrorInvalidValue;
+    if (!encode_tmap(&tmQpe, a.q_pe, 2, pdims, pstr, qpebox, 64)) return cudaErrorInvalidValue;
     // The cache holds sum(ctx) <= B * max_ctx rows; cu_ctx lives on the
     // device, so the map is declared with the bound and every box is clamped
     // inside its own sequence (chunk_base).
     const uint64_t cdims[2] = {(uint64_t)W, (uint64_t)a.B * (uint64_t)a.max_ctx};
     const uint64_t cstr[1] = {(uint64_t)W * 2};
     if (!encode_tmap(&tmC, a.cache, 2, cdims, cstr, cbox)) return cudaErrorInvalidValue;
+    if (!encode_tmap(&tmCr, a.cache, 2, cdims, cstr, rbox, 64)) return cudaErrorInvalidValue;
     // epilogue stores: fp32 partials (as bf16 pairs) and the bf16 latent output,
     // 32 rows x 128 bytes per box
     CUtensorMap tmPO, tmOL;
@@ -817,7 +820,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
       if (ea != cudaSuccess) return ea;
     }
     dim3 grid(2 * a.n_units, 1, (a.h + 127) / 128);
-    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, tmPO, tmOL, p);
+    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, tmCr, tmPO, tmOL, p);
     count_launches();
   }
   stage_event(2, st);

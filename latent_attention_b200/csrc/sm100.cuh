@@ -260,6 +260,16 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return make_desc(saddr, 16, 1024);
 }
 
+// K-major operand tile written by a TMA box {32 elements of K, rows} with
+// 64-byte swizzle (layout type 4): 8-row groups are 512 bytes apart; the
+// second 16-element K step starts 32 bytes in.
+__device__ __forceinline__ uint64_t desc_kmajor_sw64(uint32_t saddr) {
+  uint64_t d = make_desc(saddr, 16, 512);
+  d &= ~((uint64_t)7 << 61);
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+
 // MN-major operand: 64 MN-elements per 128-byte row, rows = K.  8 K-rows
 // form a 1024-byte group (stride between K groups = 1024); consecutive
 // 64-element MN blocks are `mn_block_bytes` apart.
@@ -503,9 +513,10 @@ __device__ __forceinline__ void unpack_f16(uint32_t v, float& lo, float& hi) {
 
 }  // namespace sm100
 
-// Host: encode a 2D/3D tiled tensor map (bf16, 128-byte swizzle, zero fill).
-// dims/strides innermost first; strides in bytes for dims 1..rank-1.
+// Host: encode a 2D/3D tiled tensor map (bf16, zero fill) with a 128-byte,
+// 64-byte or no swizzle (swizzle_bytes 128, 64 or 0).  dims/strides innermost
+// first; strides in bytes for dims 1..rank-1.
 bool encode_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                 const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128 = true);
+                 const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes = 128);
 
 }  // namespace mla

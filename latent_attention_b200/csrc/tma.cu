@@ -29,7 +29,7 @@ EncodeFn get_encode() {
 }  // namespace
 
 bool encode_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                 const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128) {
+                 const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
   EncodeFn fn = get_encode();
   if (!fn) return false;
   cuuint64_t d[5], s[4];
@@ -42,7 +42,9 @@ bool encode_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
   }
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
                   d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                        : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
