@@ -74,17 +74,19 @@ constexpr int R = 512, DR = 64, W = R + DR;      // latent, rope, cache row widt
 constexpr int QPE_BOX = 128 * 32 * 2;            // 128 heads x this CTA's 32 rope dims
 constexpr int CBOX = NT * 64 * 2;                // 64 tokens x 64 dims bf16
 constexpr int RBOX = NT * 32 * 2;                // 64 tokens x this CTA's 32 rope dims
-constexpr int NSTAGE = 5;                        // chunk ring
-constexpr int NSLOT = 2;                         // score slots
+constexpr int NSTAGE = 4;                        // chunk ring
+constexpr int NSLOT = 2;                         // score slots (TMEM)
+constexpr int NGRP = 2;                          // softmax groups, taking chunks in turn
+constexpr int NSB = NGRP % 2 ? 2 * NGRP : NGRP;  // score barriers: chunk g uses g % NSB
 constexpr int XBUF = 128 * NT * 2;               // one chunk's fp16 partial scores, 16 KB
 constexpr int PBUF = 128 * NT * 2;               // one chunk's P (bf16), 16 KB
 constexpr int OFF_QPE = 0;                               // rope query half, 8 KB
-constexpr int OFF_X = OFF_QPE + QPE_BOX;                 // exchange buffer
-constexpr int OFF_P = OFF_X + XBUF;                      // P buffer
-constexpr int OFF_C = OFF_P + PBUF;                      // 40 KB
+constexpr int OFF_X = OFF_QPE + QPE_BOX;                 // exchange buffers, one per group
+constexpr int OFF_P = OFF_X + NGRP * XBUF;               // P buffers, one per group
+constexpr int OFF_C = OFF_P + NGRP * PBUF;               // 72 KB
 constexpr int STAGE = 4 * CBOX + RBOX;                   // 36 KB
 constexpr int SMEM_BYTES = OFF_C + NSTAGE * STAGE + 1024;
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 128 + 128 * NGRP;
 constexpr int PREFETCH = 4;                              // chunks prefetched to L2
 constexpr uint32_t IDESC_S = idesc_bf16(128, NT);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, 0, 1);
@@ -148,11 +150,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                        const __grid_constant__ DecTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full, qt_full, q_free, c_full[NSTAGE], c_empty[NSTAGE],
-      s_full[NSLOT], s_free[NSLOT], x_full[2], x_empty[2], p_full, pv_done[2], o_done, o_free,
-      ref_ready[2];
+      s_full[NSB], s_free[NSB], x_full[NGRP], x_empty[NGRP], p_full[NGRP], pv_done[NGRP],
+      o_done, o_free, ref_ready[NGRP];
   __shared__ int epi_count;                    // epilogue warps done, all segments
   __shared__ float m_hand[128];                // reference max after the last chunk
-  __shared__ float fin_m[128], fin_l[128];      // group 1's state at a segment's end
+  __shared__ float fin_m[NGRP - 1][128], fin_l[NGRP - 1][128];  // groups 1.. at a segment's end
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag, seq_lo, seq_hi;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -172,37 +174,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     seq_lo = seq_at(cu, p.B, sl.r0);
     seq_hi = seq_at(cu, p.B, sl.r1 - 1) + 1;
     mbar_init(&q_full, 1);
-    mbar_init(&qt_full, 4);         // softmax group 1 stored the TMEM query part
+    mbar_init(&qt_full, 4);         // the last softmax group stored the TMEM query part
     mbar_init(&q_free, 1);          // the last S of a segment completed
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&c_full[s], 1);
       mbar_init(&c_empty[s], 1);
     }
-    for (int s = 0; s < NSLOT; ++s) {
+    for (int s = 0; s < NSB; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 4);     // the chunk's softmax group loaded S_g
     }
-    // The exchange buffer and the P buffer hold one chunk at a time, but
-    // their barriers come in pairs by chunk parity (phase g >> 1 of barrier
-    // g & 1), so that no waiter ever looks for a phase two ahead of the
-    // current one (a parity wait would take the older phase for it).
-    // x_full[x] counts the bytes of the peer's partial scores of a chunk
-    // (armed for chunks 0 and 1 here, then for chunk g + 2 by the group that
-    // has seen chunk g arrive); x_empty[x] completes when the peer's group has
-    // read this CTA's partial scores; pv_done[x] when PV_g has run.  p_full
-    // (P_g written) is waited for in chunk order by the MMA warp alone.
-    for (int x = 0; x < 2; ++x) {
+    // Chunk g uses the exchange buffer, the P buffer and the barriers of
+    // its group x = g % NGRP (phase g / NGRP; the score barriers likewise by
+    // g % NSB), so that every barrier is waited on by one party, in order,
+    // and no waiter ever looks for a phase two ahead of the current one (a
+    // parity wait would take the older phase for it).  x_full[x] counts the
+    // bytes of the peer's partial scores of a chunk (armed for the first
+    // NGRP chunks here, then for chunk g + NGRP by the group that has seen
+    // chunk g arrive); x_empty[x] completes when the peer's group has read
+    // this CTA's partial scores of the buffer; p_full[x] when P_g is written;
+    // pv_done[x] when PV_g has run.
+    for (int x = 0; x < NGRP; ++x) {
       mbar_init(&x_full[x], 1);
       mbar_arrive_expect_tx(&x_full[x], XBUF);
       mbar_init(&x_empty[x], 4);
+      mbar_init(&p_full[x], 4);
       mbar_init(&pv_done[x], 1);
     }
-    mbar_init(&p_full, 4);
     epi_count = 0;
     mbar_init(&o_done, 1);          // the last PV of a segment completed
     mbar_init(&o_free, 4);          // softmax group 0 has read O out of TMEM
-    mbar_init(&ref_ready[0], 4);    // a softmax group published chunk g's reference
-    mbar_init(&ref_ready[1], 4);
+    for (int x = 0; x < NGRP; ++x)
+      mbar_init(&ref_ready[x], 4);  // a softmax group published chunk g's reference
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -215,8 +218,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tbase = tmem_base;
   const int b0 = seq_lo, b1 = seq_hi;
-  // softmax groups: warps 4..7 (group 0) and 8..11 (group 1)
-  const int sm_wg = (warp >= 4 && warp < 8) ? 0 : (warp >= 8 ? 1 : -1);
+  // softmax groups: warps 4 + 4x .. 7 + 4x (group x)
+  const int sm_wg = warp >= 4 ? (warp - 4) >> 2 : -1;
 
   if (warp == 0) {
     // ---------------- the chunk ring, L2 prefetch
@@ -307,17 +310,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // PV first: its completion frees the chunk's stage
         if (gp < gs) {
           const int st = gp % NSTAGE;
-          if (mbar_test(&p_full, gp & 1) &&
+          if (mbar_test(&p_full[gp % NGRP], (gp / NGRP) & 1) &&
               (cp.j != 0 || cp.kk == 0 || mbar_test(&o_free, (cp.kk - 1) & 1))) {
             tc_fence_after();
             const uint64_t dv = desc_mnmajor_sw128(smem_u32(smem + OFF_C + st * STAGE), CBOX);
-            const uint64_t dp = desc_kmajor_sw128(smem_u32(smem + OFF_P));
+            const uint64_t dp = desc_kmajor_sw128(smem_u32(smem + OFF_P + (gp % NGRP) * PBUF));
 #pragma unroll
             for (int k = 0; k < NT / 16; ++k)
               mma_bf16(tbase + TM_O, dp + (uint64_t)((k * 32) >> 4),
                        dv + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV, (cp.j | k) != 0);
             mma_commit(&c_empty[st]);
-            mma_commit(&pv_done[gp & 1]);
+            mma_commit(&pv_done[gp % NGRP]);
             if (cp.j == cp.s.nch - 1) mma_commit(&o_done);
             ++gp;
             cp.next(cu, b0, b1, p.max_ctx, sl, u);
@@ -326,10 +329,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         if (!cs.done) {
           const int st = gs % NSTAGE, sls = gs % NSLOT;
+          const int sb = gs % NSB, sbf = (gs - NSLOT + NSB) % NSB;   // S_gs, S_{gs-2} barriers
           const uint32_t d = tbase + TM_S + sls * NT;
           const uint64_t dc = desc_kmajor_sw128(smem_u32(smem + OFF_C + st * STAGE));
           if ((cs.j != 0 || (mbar_test(&q_full, cs.kk & 1) && mbar_test(&qt_full, cs.kk & 1))) &&
-              (gs < NSLOT || mbar_test(&s_free[sls], ((gs / NSLOT) - 1) & 1)) &&
+              (gs < NSLOT || mbar_test(&s_free[sbf], ((gs - NSLOT) / NSB) & 1)) &&
               mbar_test(&c_full[st], (gs / NSTAGE) & 1)) {
             tc_fence_after();
             // partial S_gs over this CTA's dims: its latent half (query in
@@ -344,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k = 0; k < 2; ++k)
               mma_bf16(d, dq + (uint64_t)((k * 32) >> 4), dr + (uint64_t)((k * 32) >> 4), IDESC_S, 1);
-            mma_commit(&s_full[sls]);
+            mma_commit(&s_full[sb]);
             if (cs.j == cs.s.nch - 1) mma_commit(&q_free);
             ++gs;
             cs.next(cu, b0, b1, p.max_ctx, sl, u);
@@ -386,7 +390,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const uint32_t x_mine = smem_u32(smem + OFF_X) + r * 16;
     const uint32_t x_peer = mapa_shared(x_mine, rank ^ 1u);
     const uint32_t p_row = smem_u32(smem + OFF_P) + r * 128;
-    // the peer's x_full / x_empty barriers (those of parity x 8 bytes further)
+    // the peer's x_full / x_empty barriers (those of group x 8x bytes further)
     const uint32_t peer_x_full = mapa_shared(smem_u32(&x_full[0]), rank ^ 1u);
     const uint32_t peer_x_empty = mapa_shared(smem_u32(&x_empty[0]), rank ^ 1u);
     bool ok = true;
@@ -395,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int g0 = 0; !c.done; c.next_seg(cu, b0, b1, p.max_ctx, sl, u)) {
       const Seg s = c.s;
       const int kk = c.kk;
-      if (sm_wg == 1 && ok) {   // this CTA's latent half of the head's query into TMEM
+      if (sm_wg == NGRP - 1 && ok) {   // this CTA's latent half of the head's query into TMEM
         // two rounds of 16 loads (the first issued before the wait for the
         // previous segment's last S), each stored as 64 TMEM columns
         const uint4* src =
@@ -434,9 +438,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; ok && j < s.nch; ++j) {
         const int g = g0 + j;
-        if ((g & 1) != sm_wg) continue;
-        const int sls = g % NSLOT, xs = g & 1;   // score slot; the group's hand-over slot
-        if (!warp_wait(&s_full[sls], (g / NSLOT) & 1, abort_v, p.status)) { ok = false; break; }
+        if (g % NGRP != sm_wg) continue;
+        // score slot and barrier; this group and the previous chunk's group
+        const int sls = g % NSLOT, sb = g % NSB, xs = sm_wg, xp = (g + NGRP - 1) % NGRP;
+        const uint32_t ph = (g / NGRP) & 1, php = ((g - 1) / NGRP) & 1;   // their phases
+        if (!warp_wait(&s_full[sb], (g / NSB) & 1, abort_v, p.status)) { ok = false; break; }
         tc_fence_after();
         // this CTA's partial scores as fp16 pairs
         uint32_t hx[32];
@@ -447,27 +453,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
           tc_fence_before();      // the slot may take S_{g+2}
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s_free[sls]);
+          if (lane == 0) mbar_arrive(&s_free[sb]);
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             hx[e] = pack_f16_sat(__uint_as_float(sr[e >> 4][(2 * e) & 31]),
                                  __uint_as_float(sr[e >> 4][(2 * e + 1) & 31]));
         }
-        // into the peer's exchange buffer, once the peer has read chunk g - 1
-        // there: asynchronous stores that count their bytes on its x_full
-        if (g >= 1 &&
-            !warp_wait(&x_empty[xs ^ 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+        // into the peer's exchange buffer xs, once the peer has read chunk
+        // g - NGRP there: asynchronous stores that count their bytes on its
+        // x_full[xs]
+        if (g >= NGRP && !warp_wait(&x_empty[xs], ph ^ 1, abort_v, p.status)) {
           ok = false;
           break;
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          st_async_v4(x_peer + k * 2048, peer_x_full + 8 * xs, hx[4 * k], hx[4 * k + 1],
+          st_async_v4(x_peer + xs * XBUF + k * 2048, peer_x_full + 8 * xs, hx[4 * k], hx[4 * k + 1],
                       hx[4 * k + 2], hx[4 * k + 3]);
         // the peer's partial scores of chunk g; then x_full[xs] is armed for
-        // chunk g + 2, whose bytes the peer sends only after chunk g + 1 has
-        // been read here, which follows this group's reading of chunk g
-        if (!warp_wait_cluster(&x_full[xs], (g >> 1) & 1, abort_v, p.status)) {
+        // chunk g + NGRP, whose bytes the peer sends only after chunk
+        // g + NGRP - 1 has been read here, which follows this group's reading
+        // of chunk g
+        if (!warp_wait_cluster(&x_full[xs], ph, abort_v, p.status)) {
           ok = false;
           break;
         }
@@ -475,7 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         float sv[NT];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint4 v = ld_shared_v4(x_mine + k * 2048);
+          const uint4 v = ld_shared_v4(x_mine + xs * XBUF + k * 2048);
           const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -486,7 +493,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             sv[8 * k + 2 * i + 1] = a1 + b1;
           }
         }
-        __syncwarp();   // the values are summed: the buffer may take chunk g + 1
+        __syncwarp();   // the values are summed: the buffer may take chunk g + NGRP
         if (lane == 0) mbar_arrive_cluster_relaxed(peer_x_empty + 8 * xs);
         // column i holds token base + i; chunk j owns tokens [t0 + 64j, t0 + tcount)
         const int base = chunk_base(s.n, s.t0, j) - s.t0;
@@ -507,7 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // in order across segments, where the reference itself starts afresh.
         float m_prev = -INFINITY;
         if (g > 0) {
-          if (!warp_wait(&ref_ready[xs ^ 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+          if (!warp_wait(&ref_ready[xp], php, abort_v, p.status)) {
             ok = false;
             break;
           }
@@ -538,16 +545,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           w[e] = pack_bf16(p0, p1);
         }
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        // PV_{g-1} has run: it no longer reads the P buffer, and O holds the
-        // segment's sum through chunk j-1 at reference m_prev -- rescale it
-        // when this chunk moved the reference.
-        if (g >= 1 &&
-            !warp_wait(&pv_done[xs ^ 1], ((g - 1) >> 1) & 1, abort_v, p.status)) {
+        // PV_{g-NGRP} has run: this group's P buffer is free (this wait, on
+        // every chunk and in order, also completes PV_{g-NGRP-1}, so the one
+        // below never sees a barrier two phases behind).
+        if (g >= NGRP && !warp_wait(&pv_done[xs], ph ^ 1, abort_v, p.status)) {
           ok = false;
           break;
         }
+        // O holds the segment's sum through chunk j-1 at reference m_prev:
+        // rescale it when this chunk moved the reference (PV_{g-1} must have
+        // run).
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
           const float alpha = ex2(m_prev - m_new);
+          if (!warp_wait(&pv_done[xp], php, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < 8; ++cc) {
@@ -560,35 +573,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           }
           tmem_wait_st();
         }
-        // P_g into the P buffer
+        // P_g into this group's P buffer
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          st_shared_v4(p_row + ((k ^ (r & 7)) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
-                       w[4 * k + 3]);
+          st_shared_v4(p_row + xs * PBUF + ((k ^ (r & 7)) << 4), w[4 * k], w[4 * k + 1],
+                       w[4 * k + 2], w[4 * k + 3]);
         fence_proxy_async();
         tc_fence_before();        // the O rescale above happens before PV_g
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full);
+        if (lane == 0) mbar_arrive(&p_full[xs]);
       }
       g0 += s.nch;
-      // Segment end.  Both groups' sums at the last chunk's reference
-      // (references never decrease, so that is the larger of the two).
-      // Group 1 hands over through fin_*, once group 0 has finished the
-      // previous segment (o_free), which it does only after reading them.
-      // Both groups pass one barrier per segment, also after a failed wait.
-      if (sm_wg == 1) {
-        if (ok && kk > 0 && !warp_wait(&o_free, (kk - 1) & 1, abort_v, p.status)) ok = false;
-        fin_m[r] = m_ref;
-        fin_l[r] = l;
-        named_barrier_sync(1, 256);
-      } else {
-        named_barrier_sync(1, 256);
+      // Segment end.  Every group's sum at its last chunk's reference
+      // (references never decrease, so the largest is the row's).  The other
+      // groups hand over through fin_*; every softmax thread passes the two
+      // barriers (after the writes, after group 0's reads) on every path.
+      if (sm_wg > 0) {
+        fin_m[sm_wg - 1][r] = m_ref;
+        fin_l[sm_wg - 1][r] = l;
+      }
+      named_barrier_sync(1, 128 * NGRP);
+      float m_last = m_ref, l_tot = 0.f;
+      if (sm_wg == 0) {
+#pragma unroll
+        for (int x = 0; x < NGRP - 1; ++x) m_last = fmaxf(m_last, fin_m[x][r]);
+        l_tot = l > 0.f ? l * ex2(m_ref - m_last) : 0.f;
+#pragma unroll
+        for (int x = 0; x < NGRP - 1; ++x) {
+          const float lx = fin_l[x][r];
+          l_tot += lx > 0.f ? lx * ex2(fin_m[x][r] - m_last) : 0.f;
+        }
+      }
+      named_barrier_sync(1, 128 * NGRP);
+      if (sm_wg == 0) {
         if (ok && !warp_wait(&o_done, kk & 1, abort_v, p.status)) ok = false;
         if (ok) {
-          const float m1 = fin_m[r], l1 = fin_l[r];
-          const float m_last = fmaxf(m_ref, m1);
-          const float l_tot = (l > 0.f ? l * ex2(m_ref - m_last) : 0.f) +
-                              (l1 > 0.f ? l1 * ex2(m1 - m_last) : 0.f);
           const float inv = 1.f / l_tot;
           tc_fence_after();
           // This warp's 32 rows go out through the latent boxes of the
