@@ -98,6 +98,7 @@ constexpr int EPI_BOX = 32 * 128;             // epilogue staging: 32 rows of 12
 
 struct DecTcParams {
   const int32_t* cu_ctx;
+  const uint8_t* cache;        // [sum ctx, 576] bf16 rows (for L2 prefetch)
   const __nv_bfloat16* q_lat;  // [B, h, 512]
   int B, h, max_ctx;
   int n_units, min_len;        // CTA pairs; shortest slice of the token stream
@@ -227,11 +228,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       tma_prefetch(&tmQ);
       tma_prefetch(&tmC);
       tma_prefetch(&tmCr);
-      // this CTA's boxes of chunk j of segment s into L2
+      // chunk j of segment s into L2: its rows are contiguous in the cache
+      // (the rows its boxes read, less any before row 0); this CTA takes
+      // half of the bytes
       auto prefetch = [&](const Seg& s, int j) {
         const int y = (int)s.start + chunk_base(s.n, s.t0, j);
-        for (int a = 0; a < 4; ++a) tma_prefetch_l2_2d(&tmC, dim0 + 64 * a, y);
-        tma_prefetch_l2_2d(&tmCr, R + 32 * (int)rank, y);
+        const int y0 = max(y, 0);
+        const uint32_t half = (uint32_t)(y + NT - y0) * (W * 2 / 2);   // 576 bytes per row
+        bulk_prefetch_l2(p.cache + (uint64_t)y0 * (W * 2) + rank * half, half);
       };
       // this CTA's latent half of a segment's query rows into L2
       auto prefetch_q = [&](const Seg& s) {
@@ -822,6 +826,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
     if (!encode_tmap(&tmOL, a.o_lat, 2, oldims, olstr, obox)) return cudaErrorInvalidValue;
     DecTcParams p{};
     p.cu_ctx = a.cu_ctx;
+    p.cache = reinterpret_cast<const uint8_t*>(a.cache);
     p.q_lat = reinterpret_cast<const __nv_bfloat16*>(a.q_lat);
     p.B = a.B;
     p.h = a.h;

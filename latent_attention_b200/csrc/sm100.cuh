@@ -396,6 +396,14 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, 
                : "memory");
 }
 
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned start) into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
