@@ -62,6 +62,7 @@ struct TcGemmParams {
   uint32_t* status;
 };
 
+template <int TBN>
 __device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& bi, int& s,
                                             int& m0, int& n0) {
   bi = t / p.per_batch;
@@ -76,10 +77,11 @@ __device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& b
   const int gm = min(G, p.tiles_m - g * G);               // rows of this group
   const int in = local - g * G * tn;
   m0 = (g * G + in % gm) * BM;
-  n0 = (in / gm) * BN;
+  n0 = (in / gm) * TBN;
 }
 
-// Epilogue of one 128 x BN tile; this thread owns output row m0 + row.
+// Epilogue of one 128 x TBN tile; this thread owns output row m0 + row.
+template <int TBN = BN>
 __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSeg& e, int bi,
                                               int m0, int n0, int row, uint32_t taddr,
                                               const CUtensorMap* tmO, uint32_t stg, int& gidx) {
@@ -96,7 +98,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out) + (int64_t)bi * p.sOut;
   const __nv_bfloat16* gamma = reinterpret_cast<const __nv_bfloat16*>(e.gamma);
 #pragma unroll 1
-  for (int g = 0; g < BN / 64; ++g) {
+  for (int g = 0; g < TBN / 64; ++g) {
     const int nl = n0 + g * 64;
     if (nl >= e.ncols) break;  // uniform over the warp
     uint32_t r0[32], r1[32];
@@ -184,9 +186,13 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
       }
     }
   }
-  if (e.ssq_out && row_ok && n0 < e.norm_cols) e.ssq_out[(n0 / BN) * e.ssq_ld + m] = ssq;
+  if (e.ssq_out && row_ok && n0 < e.norm_cols) e.ssq_out[(n0 / TBN) * e.ssq_ld + m] = ssq;
 }
 
+// TBN: tile width (256 in general; 512 for one-wave batched products whose
+// whole output row fits one tile, using all of TMEM for one accumulator; 128
+// for batched products of at most 128 columns), TST: ring stages.
+template <int TBN, int TST>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB0,
@@ -194,8 +200,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmO0,
                    const __grid_constant__ CUtensorMap tmO1,
                    const __grid_constant__ TcGemmParams p) {
+  constexpr int kBBytes = TBN * BK * 2;
+  constexpr int kStage = A_BYTES + kBBytes;
+  constexpr int kOffOut = TST * kStage;
+  constexpr int kNBuf = TBN == 512 ? 1 : 2;              // TMEM accumulators
+  constexpr uint32_t kTmem = TBN == 512 ? 512u : 2u * TBN;
+  constexpr int kNMma = TBN == 512 ? 2 : 1;              // MMAs of N = TBN / kNMma per K step
+  constexpr uint32_t kIdesc = idesc_bf16(BM, TBN / kNMma);
+  constexpr uint32_t kIdescMN = idesc_bf16(BM, TBN / kNMma, 0, 1);
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2];
+  __shared__ __align__(8) uint64_t full[TST], empty[TST], tfull[2], tempty[2];
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -204,7 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile int* abort_v = &abort_flag;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < TST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (p.nseg > 1) tma_prefetch(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base, TMEM_COLS);
+    tmem_alloc(&tmem_base, kTmem);
     tc_fence_before();
   }
   __syncthreads();
@@ -235,23 +249,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
         int bi, s, m0, n0;
-        tile_coords(p, t, bi, s, m0, n0);
+        tile_coords<TBN>(p, t, bi, s, m0, n0);
         const CUtensorMap* tmB = s ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_v, p.status)) goto done;
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t* sa = smem + stage * kStage;
+          mbar_arrive_expect_tx(&full[stage], kStage);
           if (p.a_batch_inner)
             tma_load_3d(sa, &tmA, kb * BK, bi, m0, &full[stage]);
           else
             tma_load_3d(sa, &tmA, kb * BK, m0, bi, &full[stage]);
           if (p.b_mn) {
-            for (int q = 0; q < BN / 64; ++q)
+            for (int q = 0; q < TBN / 64; ++q)
               tma_load_3d(sa + A_BYTES + q * BMN_BOX, tmB, n0 + 64 * q, kb * BK, bi, &full[stage]);
           } else {
-            tma_load_3d(sa + A_BYTES, tmB, kb * BK, n0, bi, &full[stage]);
+            for (int q = 0; q < kNMma; ++q)    // boxes of at most 256 rows
+              tma_load_3d(sa + A_BYTES + q * (kBBytes / kNMma), tmB, kb * BK,
+                          n0 + q * (TBN / kNMma), bi, &full[stage]);
           }
-          if (++stage == STAGES) {
+          if (++stage == TST) {
             stage = 0;
             phase ^= 1;
           }
@@ -264,29 +280,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
-        const int buf = local & 1;
-        const uint32_t tph = (local >> 1) & 1;
+        const int buf = local % kNBuf;
+        const uint32_t tph = (local / kNBuf) & 1;
         if (!mbar_wait(&tempty[buf], tph ^ 1, abort_v, p.status)) goto done;
         tc_fence_after();
-        const uint32_t d = tbase + buf * BN;
+        const uint32_t d = tbase + buf * TBN;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_v, p.status)) goto done;
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * kStage);
           const uint32_t sb = sa + A_BYTES;
           if (p.b_mn) {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
-              mma_bf16(d, desc_kmajor_sw128(sa + k * 32),
-                       desc_mnmajor_sw128(sb + k * 16 * 128, BMN_BOX), IDESC_BMN, (kb | k) != 0);
+#pragma unroll
+              for (int q = 0; q < kNMma; ++q)
+                mma_bf16(d + q * (TBN / kNMma), desc_kmajor_sw128(sa + k * 32),
+                         desc_mnmajor_sw128(sb + q * (kBBytes / kNMma) + k * 16 * 128, BMN_BOX),
+                         kIdescMN, (kb | k) != 0);
           } else {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
-              mma_bf16(d, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), IDESC,
-                       (kb | k) != 0);
+#pragma unroll
+              for (int q = 0; q < kNMma; ++q)
+                mma_bf16(d + q * (TBN / kNMma), desc_kmajor_sw128(sa + k * 32),
+                         desc_kmajor_sw128(sb + q * (kBBytes / kNMma) + k * 32), kIdesc,
+                         (kb | k) != 0);
           }
           mma_commit(&empty[stage]);
-          if (++stage == STAGES) {
+          if (++stage == TST) {
             stage = 0;
             phase ^= 1;
           }
@@ -297,19 +319,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const uint32_t stg = smem_u32(smem + OFF_OUT + quad * 2 * OUT_BOX);
+    const uint32_t stg = smem_u32(smem + kOffOut + quad * 2 * OUT_BOX);
     int gidx = 0;
     int local = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
-      const int buf = local & 1;
-      const uint32_t tph = (local >> 1) & 1;
+      const int buf = local % kNBuf;
+      const uint32_t tph = (local / kNBuf) & 1;
       if (!warp_wait(&tfull[buf], tph, abort_v, p.status)) break;
       tc_fence_after();
       int bi, s, m0, n0;
-      tile_coords(p, t, bi, s, m0, n0);
-      epilogue_tile(p, p.seg[s], bi, m0, n0, row,
-                    tbase + ((uint32_t)(quad * 32) << 16) + buf * BN, s ? &tmO1 : &tmO0, stg,
-                    gidx);
+      tile_coords<TBN>(p, t, bi, s, m0, n0);
+      epilogue_tile<TBN>(p, p.seg[s], bi, m0, n0, row,
+                         tbase + ((uint32_t)(quad * 32) << 16) + buf * TBN, s ? &tmO1 : &tmO0,
+                         stg, gidx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -321,7 +343,7 @@ done:
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, TMEM_COLS);
+    tmem_dealloc(tbase, kTmem);
   }
 }
 
@@ -521,6 +543,21 @@ bool tc_gemm_supported(const GemmArgs& a, int dtype) {
   return true;
 }
 
+namespace {
+template <int TBN, int TST>
+cudaError_t launch_single(int grid, const CUtensorMap& tmA, const CUtensorMap (&tmB)[2],
+                          const CUtensorMap (&tmO)[2], const TcGemmParams& p, cudaStream_t st) {
+  constexpr int smem = TST * (A_BYTES + TBN * BK * 2) + 4 * 2 * OUT_BOX + 1024;
+  static_assert(smem <= 227 * 1024, "shared memory");
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc_kernel<TBN, TST>, smem, smem_set);
+  if (ea != cudaSuccess) return ea;
+  gemm_tc_kernel<TBN, TST><<<grid, NTHREADS, smem, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);
+  count_launches();
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   CUtensorMap tmA, tmB[2];
   const uint64_t nb = (uint64_t)a.batch;
@@ -545,7 +582,17 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   // faster on single CTAs
   const bool pair = a.batch == 1 && !a.b_mn && !a.a_batch_inner && a.M >= 512 && a.K >= 1024;
   const int bm = pair ? BM2 : BM;
-  const int b_rows = pair ? 128 : BN;     // B rows per CTA and stage
+  // Batched products whose rows fit one 128-row tile (the absorbed decode's
+  // per-head products, M = the sequences): the whole output row of a batch
+  // entry in one tile -- 512 columns in all of TMEM, or 128 -- so that one
+  // wave of CTAs covers the batch and no B rows beyond the product are read.
+  int tbn = BN;
+  if (!pair && a.batch > 1 && a.M <= BM && a.nseg == 1) {
+    const int n = a.seg[0].ncols;
+    if (n <= 128) tbn = 128;
+    else if (n > BN && n <= 512) tbn = 512;
+  }
+  const int b_rows = pair ? 128 : (tbn < 256 ? tbn : 256);   // B rows per CTA and box
   TcGemmParams p{};
   p.M = a.M;
   p.K = a.K;
@@ -569,7 +616,7 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
     }
     if (!encode_tmap(&tmB[s], a.Bm[s], 3, dims, strides, box)) return cudaErrorInvalidValue;
     p.seg[s] = a.seg[s];
-    p.tiles_n[s] = (int)((n + BN - 1) / BN);
+    p.tiles_n[s] = (int)((n + tbn - 1) / tbn);
     p.per_batch += p.tiles_m * p.tiles_n[s];
   }
   if (a.nseg == 1) {
@@ -611,15 +658,10 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
     count_launches();
     return cudaGetLastError();
   }
-  static std::atomic<uint64_t> smem_set{0};
-  {
-    const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc_kernel, SMEM_BYTES, smem_set);
-    if (ea != cudaSuccess) return ea;
-  }
   const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
-  gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);
-  count_launches();
-  return cudaGetLastError();
+  if (tbn == 512) return launch_single<512, 2>(grid, tmA, tmB, tmO, p, st);
+  if (tbn == 128) return launch_single<128, 6>(grid, tmA, tmB, tmO, p, st);
+  return launch_single<BN, STAGES>(grid, tmA, tmB, tmO, p, st);
 }
 
 }  // namespace mla
