@@ -63,3 +63,10 @@ def test_other_prefill_workloads_are_timed_beside_the_headline():
                                          "kimi_prefill"}
     for n in bench.PREFILL_OTHERS:
         assert WORKLOADS[n].kind == "prefill"
+
+
+def test_reference_arm_and_cpu_baseline_time_the_same_oracle_sample():
+    rows = bench.oracle_rows(4096)
+    assert rows[:3] == [0, 16, 32] and rows[-1] == 4095 and len(rows) == 257
+    assert bench.oracle_rows(64) == [0, 16, 32, 48, 63]
+    assert bench.oracle_rows(17) == [0, 16]
