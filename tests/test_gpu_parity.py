@@ -143,8 +143,8 @@ def test_prefill_full_size_sampled_rows(cuda, name):
                                     ("directq_prefill", 1000)])
 def test_prefill_ragged_rows_on_cta_pairs(cuda, name, T):
     """Row counts that are not a multiple of the 256-row tiles of the CTA-pair
-    projections (K >= 1024): at 777 rows the last tile's second CTA holds no
-    row, at 1000 it holds 104 of its 128."""
+    projections: at 777 rows the last tile's second CTA holds no row, at 1000
+    it holds 104 of its 128."""
     cfg = W[name].cfg
     inp = make_prefill_inputs(cfg, 1, T, seed=4)
     layer, out, _ = run_prefill(cfg, inp, latent=False)
@@ -153,6 +153,25 @@ def test_prefill_ragged_rows_on_cta_pairs(cuda, name, T):
     ref = oracle.prefill(cfg, inp, rows=rows)
     got = out[:, torch.as_tensor(rows)]
     assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
+
+
+def test_prefill_one_head_many_row_tiles(cuda):
+    """One head: the kv up-projection (K = 512), the q up-projection (K = 256)
+    and o_proj (K = 128) are one 256-column tile wide and 313 row tiles deep,
+    so every CTA takes two or three tiles of different rows, and the last
+    tile is ragged."""
+    cfg = small_bf16(num_heads=1)
+    T = 40000
+    inp = make_prefill_inputs(cfg, 1, T, seed=6)
+    layer, out, _ = run_prefill(cfg, inp, latent=False)
+    rows = sorted(set(sample_rows(T, 16)) | {0, 255, 256, 511, 20479, 20480, T - 1})
+    ref, P = oracle.prefill(cfg, inp, rows=rows, return_parts=True)
+    got = out[:, torch.as_tensor(rows)]
+    assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
+    # every row of the kv up-projection
+    kv = f64(layer.view("kv", (1, T, 1, cfg.qk_nope_head_dim + cfg.v_head_dim)))
+    assert oracle.max_rel_err(kv[..., :cfg.qk_nope_head_dim], P["k_nope"]) <= TOL[cfg.dtype]
+    assert oracle.max_rel_err(kv[..., cfg.qk_nope_head_dim:], P["v"]) <= TOL[cfg.dtype]
 
 
 # --------------------------------------------------------------------------
