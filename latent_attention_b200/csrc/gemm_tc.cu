@@ -34,16 +34,10 @@ using namespace sm100;
 
 constexpr int BM = 128, BN = kTcTileN, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 // Output staging for TMA stores: per epilogue warp two 32-row x 64-column
 // bf16 boxes (4 KB each), 128-byte swizzled.
 constexpr int OUT_BOX = 32 * 64 * 2;
-constexpr int OFF_OUT = STAGES * STAGE_BYTES;
-constexpr int SMEM_BYTES = OFF_OUT + 4 * 2 * OUT_BOX + 1024;
 constexpr int NTHREADS = 192;
-constexpr uint32_t IDESC = idesc_bf16(BM, BN);
-constexpr uint32_t IDESC_BMN = idesc_bf16(BM, BN, 0, 1);
 constexpr int BMN_BOX = 64 * BK * 2;       // one 64-column MN-major box of B
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
@@ -81,6 +75,9 @@ __device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& b
 }
 
 // Epilogue of one 128 x TBN tile; this thread owns output row m0 + row.
+// Columns go out in groups of 64 (a TMA store each); a last group narrower
+// than 64 (TBN = 224) is stored directly so that no store reaches the next
+// tile's columns.
 template <int TBN = BN>
 __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSeg& e, int bi,
                                               int m0, int n0, int row, uint32_t taddr,
@@ -98,8 +95,9 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out) + (int64_t)bi * p.sOut;
   const __nv_bfloat16* gamma = reinterpret_cast<const __nv_bfloat16*>(e.gamma);
 #pragma unroll 1
-  for (int g = 0; g < TBN / 64; ++g) {
+  for (int g = 0; g < (TBN + 63) / 64; ++g) {
     const int nl = n0 + g * 64;
+    const int tw = min(64, TBN - g * 64);   // columns of this group inside the tile
     if (nl >= e.ncols) break;  // uniform over the warp
     uint32_t r0[32], r1[32];
     tmem_ld32(taddr + g * 64, r0);
@@ -154,7 +152,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
       for (int i = 0; i < 64; ++i)
         if (i < lim) v[i] *= __bfloat162float(gamma[nl + i]);
     }
-    if (p.tma_store) {
+    if (p.tma_store && tw == 64) {
       // this warp's 32 rows x 64 columns through shared memory, one TMA store
       const int lane = row & 31;
       const uint32_t sb = stg + (gidx & 1) * OUT_BOX;
@@ -177,7 +175,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmParams& p, const EpiSe
       ++gidx;
     } else if (row_ok) {
       __nv_bfloat16* dst = out + (int64_t)m * e.ldo + nl;
-      const int lim = e.ncols - nl;
+      const int lim = min(e.ncols - nl, tw);
 #pragma unroll
       for (int c = 0; c < 64; c += 8) {
         if (c < lim)
@@ -354,13 +352,20 @@ done:
 // k-block), so the same shared memory holds six stages instead of four and
 // covers more load latency; each CTA's TMEM holds its 128 output rows x 256
 // columns and its own epilogue warps write them.
+//
+// The tile is 256 x TBN2 with TBN2 = 256, or 224 where that leaves fewer
+// idle CTA pairs in the last wave (o_proj at 4096 rows: 448 tiles of 256 on
+// 74 pairs are 6.05 waves, 512 of 224 are 6.92); each CTA loads TBN2 / 2
+// rows of B.
 constexpr int BM2 = 256, STAGES2 = 6;
-constexpr int HALF_BYTES = 128 * BK * 2;                  // 16 KB
-constexpr int STAGE2_BYTES = 2 * HALF_BYTES;              // A half + B half
-constexpr int OFF_OUT2 = STAGES2 * STAGE2_BYTES;          // 192 KB
-constexpr int SMEM2_BYTES = OFF_OUT2 + 4 * 2 * OUT_BOX + 1024;
-constexpr uint32_t IDESC2 = idesc_bf16(BM2, BN);
+constexpr int HALF_BYTES = 128 * BK * 2;                  // 16 KB of A per CTA and stage
+template <int TBN2>
+constexpr int stage2_bytes() { return HALF_BYTES + TBN2 / 2 * BK * 2; }   // + B half
+template <int TBN2>
+constexpr int smem2_bytes() { return STAGES2 * stage2_bytes<TBN2>() + 4 * 2 * OUT_BOX + 1024; }
+static_assert(smem2_bytes<256>() <= 227 * 1024, "shared memory");
 
+template <int TBN2>
 __device__ __forceinline__ void tile_coords2(const TcGemmParams& p, int t, int& s, int& m0,
                                              int& n0) {
   const int first = p.tiles_m * p.tiles_n[0];
@@ -371,9 +376,10 @@ __device__ __forceinline__ void tile_coords2(const TcGemmParams& p, int t, int& 
   const int gm = min(G, p.tiles_m - g * G);
   const int in = local - g * G * tn;
   m0 = (g * G + in % gm) * BM2;
-  n0 = (in / gm) * BN;
+  n0 = (in / gm) * TBN2;
 }
 
+template <int TBN2>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -381,6 +387,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     const __grid_constant__ CUtensorMap tmO0,
                     const __grid_constant__ CUtensorMap tmO1,
                     const __grid_constant__ TcGemmParams p) {
+  constexpr int kStage = stage2_bytes<TBN2>();
+  constexpr int kOffOut = STAGES2 * kStage;
+  constexpr uint32_t kIdesc = idesc_bf16(BM2, TBN2);
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[STAGES2], empty[STAGES2], tfull[2], tempty[2];
   __shared__ uint32_t tmem_base;
@@ -429,15 +438,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       uint32_t phase = 0;
       for (int t = cid; t < p.total_tiles; t += ncl) {
         int s, m0, n0;
-        tile_coords2(p, t, s, m0, n0);
+        tile_coords2<TBN2>(p, t, s, m0, n0);
         const CUtensorMap* tmB = s ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_v, p.status)) goto done;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE2_BYTES);
-          uint8_t* sa = smem + stage * STAGE2_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStage);
+          uint8_t* sa = smem + stage * kStage;
           const uint32_t fb = full0 + stage * 8;
           tma_load_3d_pair(sa, &tmA, kb * BK, m0 + 128 * (int)rank, 0, fb);
-          tma_load_3d_pair(sa + HALF_BYTES, tmB, kb * BK, n0 + 128 * (int)rank, 0, fb);
+          tma_load_3d_pair(sa + HALF_BYTES, tmB, kb * BK, n0 + TBN2 / 2 * (int)rank, 0, fb);
           if (++stage == STAGES2) {
             stage = 0;
             phase ^= 1;
@@ -456,16 +465,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t tph = (local >> 1) & 1;
         if (!mbar_wait(&tempty[buf], tph ^ 1, abort_v, p.status)) goto done;
         tc_fence_after();
-        const uint32_t d = tbase + buf * BN;
+        const uint32_t d = tbase + buf * BN;     // accumulators 256 columns apart
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_v, p.status)) goto done;
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * kStage);
           const uint32_t sb = sa + HALF_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_bf16_pair(d, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32),
-                          IDESC2, (kb | k) != 0);
+                          kIdesc, (kb | k) != 0);
           const uint32_t eb = smem_u32(&empty[stage]);
           mma_commit_pair(eb);
           mma_commit_pair(mapa_shared(eb, peer));
@@ -483,7 +492,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     // ---------------- epilogue (both CTAs): this CTA's 128 rows of each tile
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const uint32_t stg = smem_u32(smem + OFF_OUT2 + quad * 2 * OUT_BOX);
+    const uint32_t stg = smem_u32(smem + kOffOut + quad * 2 * OUT_BOX);
     int gidx = 0;
     int local = 0;
     for (int t = cid; t < p.total_tiles; t += ncl, ++local) {
@@ -492,10 +501,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       if (!warp_wait(&tfull[buf], tph, abort_v, p.status)) break;
       tc_fence_after();
       int s, m0, n0;
-      tile_coords2(p, t, s, m0, n0);
-      epilogue_tile(p, p.seg[s], 0, m0 + 128 * (int)rank, n0, row,
-                    tbase + ((uint32_t)(quad * 32) << 16) + buf * BN, s ? &tmO1 : &tmO0, stg,
-                    gidx);
+      tile_coords2<TBN2>(p, t, s, m0, n0);
+      epilogue_tile<TBN2>(p, p.seg[s], 0, m0 + 128 * (int)rank, n0, row,
+                          tbase + ((uint32_t)(quad * 32) << 16) + buf * BN, s ? &tmO1 : &tmO0,
+                          stg, gidx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
@@ -556,6 +565,19 @@ cudaError_t launch_single(int grid, const CUtensorMap& tmA, const CUtensorMap (&
   count_launches();
   return cudaGetLastError();
 }
+
+template <int TBN2>
+cudaError_t launch_pair(int pairs, const CUtensorMap& tmA, const CUtensorMap (&tmB)[2],
+                        const CUtensorMap (&tmO)[2], const TcGemmParams& p, cudaStream_t st) {
+  constexpr int smem = smem2_bytes<TBN2>();
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc2_kernel<TBN2>, smem, smem_set);
+  if (ea != cudaSuccess) return ea;
+  gemm_tc2_kernel<TBN2><<<2 * pairs, NTHREADS, smem, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1],
+                                                            p);
+  count_launches();
+  return cudaGetLastError();
+}
 }  // namespace
 
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
@@ -592,7 +614,26 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
     if (n <= 128) tbn = 128;
     else if (n > BN && n <= 512) tbn = 512;
   }
-  const int b_rows = pair ? 128 : (tbn < 256 ? tbn : 256);   // B rows per CTA and box
+  // pair tile width: 224 instead of 256 where that cuts waves x width by at
+  // least 5 % (fewer pairs idle in the last wave; o_proj at 4096 rows: 12 %
+  // predicted, 0.663 -> 0.608 ms measured; at 16384 rows only 2 % predicted
+  // and 224 measured 3 % slower), for outputs without RoPE or RMS partials
+  // (both assume 256-column tiles)
+  int tbn2 = BN;
+  if (pair) {
+    bool plain_epi = true;
+    int64_t t256 = 0, t224 = 0;
+    const int64_t tm = (a.M + BM2 - 1) / BM2, np = num_sms() / 2;
+    for (int s = 0; s < a.nseg; ++s) {
+      plain_epi = plain_epi && !a.seg[s].cos && !a.seg[s].ssq_out;
+      t256 += tm * ((a.seg[s].ncols + 255) / 256);
+      t224 += tm * ((a.seg[s].ncols + 223) / 224);
+    }
+    const int64_t w256 = (t256 + np - 1) / np, w224 = (t224 + np - 1) / np;
+    if (plain_epi && w224 * 224 * 20 <= w256 * 256 * 19) tbn2 = 224;
+    tbn = tbn2;
+  }
+  const int b_rows = pair ? tbn2 / 2 : (tbn < 256 ? tbn : 256);   // B rows per CTA and box
   TcGemmParams p{};
   p.M = a.M;
   p.K = a.K;
@@ -649,14 +690,9 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, uint32_t* status) {
   p.sOut = a.sOut;
   p.status = status;
   if (pair) {
-    static std::atomic<uint64_t> smem2_set{0};
-    const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc2_kernel, SMEM2_BYTES, smem2_set);
-    if (ea != cudaSuccess) return ea;
     const int pairs = p.total_tiles < num_sms() / 2 ? p.total_tiles : num_sms() / 2;
-    gemm_tc2_kernel<<<2 * pairs, NTHREADS, SMEM2_BYTES, st>>>(tmA, tmB[0], tmB[1], tmO[0],
-                                                               tmO[1], p);
-    count_launches();
-    return cudaGetLastError();
+    if (tbn2 == 224) return launch_pair<224>(pairs, tmA, tmB, tmO, p, st);
+    return launch_pair<256>(pairs, tmA, tmB, tmO, p, st);
   }
   const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
   if (tbn == 512) return launch_single<512, 2>(grid, tmA, tmB, tmO, p, st);

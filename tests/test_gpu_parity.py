@@ -155,6 +155,21 @@ def test_prefill_ragged_rows_on_cta_pairs(cuda, name, T):
     assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
 
 
+def test_prefill_o_proj_on_224_column_tiles(cuda):
+    """o_proj at 4096 rows and 7000 output columns (K = 8 heads x 128): 256 x
+    224 pair tiles fill the last wave better than 256 x 256, so they are
+    used; each tile's last 32 columns go out by direct stores, and the last
+    tile column holds 56 of its 224."""
+    cfg = small_bf16(num_heads=8, hidden_size=7000)
+    T = 4096
+    inp = make_prefill_inputs(cfg, 1, T, seed=7)
+    layer, out, _ = run_prefill(cfg, inp, latent=False)
+    rows = sorted(set(sample_rows(T, 16)) | {0, 127, 128, 255, 256, 3839, 3840, T - 1})
+    ref = oracle.prefill(cfg, inp, rows=rows)
+    got = out[:, torch.as_tensor(rows)]
+    assert oracle.max_rel_err(got, ref) <= TOL[cfg.dtype]
+
+
 def test_prefill_one_head_many_row_tiles(cuda):
     """One head: the kv up-projection (K = 512), the q up-projection (K = 256)
     and o_proj (K = 128) are one 256-column tile wide and 313 row tiles deep,
