@@ -13,8 +13,9 @@
 // around does not apply).
 //
 // One CTA = (batch, head, two 128-query tiles A and B); every K/V block it
-// loads serves both tiles.  All query tiles of one head run together
-// (heaviest first), so a head's keys and values leave HBM once.  Warp roles
+// loads serves both tiles.  The CTAs of eight (sequence, head) pairs at a
+// time run together, longest first, so a head's keys and values leave HBM
+// once and the grid ends on short CTAs.  Warp roles
 // (640 threads):
 //   warp 0       TMA: Q of both tiles (once), K (one stage of 3 boxes)
 //   warp 2       TMA: V ring (2 stages of 2 boxes of 64 value columns)
@@ -54,6 +55,7 @@ constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, DV, 0, 1);   // V is MN-major
 constexpr uint32_t TM_S = 0, TM_O = 256;                   // + 128 * tile
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kHeadGroup = 8;      // (sequence, head) pairs whose CTAs are ordered together
 
 struct AttnTcParams {
   int B, T, h;           // T queries per sequence
@@ -83,9 +85,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_v = &abort_flag;
 
-  const int hh = blockIdx.y % p.h;
-  const int b = blockIdx.y / p.h;
-  const int c = p.n_pairs - 1 - blockIdx.x;          // heaviest pair first
+  // Launch order: groups of kHeadGroup (sequence, head) pairs, and inside a
+  // group all its CTAs longest first (pair c has about 2c + 2 key blocks).
+  // A group's keys and values stay in L2 while its CTAs run; longest first
+  // keeps the last CTAs of the grid short.
+  const int nbh = p.B * p.h;
+  const int grp = blockIdx.x / (p.n_pairs * kHeadGroup);
+  const int gh = min(kHeadGroup, nbh - grp * kHeadGroup);          // pairs in this group
+  const int rem = blockIdx.x - grp * p.n_pairs * kHeadGroup;
+  const int bh = grp * kHeadGroup + rem % gh;
+  const int hh = bh % p.h;
+  const int b = bh / p.h;
+  const int c = p.n_pairs - 1 - rem / gh;
   int row0, krow0, Tq, Tk, q_off;                    // this sequence's rows and lengths
   if (p.cu) {   // packed: bounds clamped to [0, total) so no store leaves the buffer
     const int s0 = min(max(p.cu[b], 0), p.total);
@@ -403,7 +414,7 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
     const cudaError_t ea = set_dynamic_smem((const void*)attn_tc_kernel, SMEM_BYTES, smem_set);
     if (ea != cudaSuccess) return ea;
   }
-  dim3 grid(p.n_pairs, a.h * a.B);
+  dim3 grid(p.n_pairs * a.h * a.B);
   attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmKV, tmKpe, p);
   count_launches();
   return cudaGetLastError();
