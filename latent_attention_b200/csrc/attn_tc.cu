@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_v = &abort_flag;
+  griddep_wait();
+  griddep_launch_dependents();
 
   // Launch order: groups of kHeadGroup (sequence, head) pairs, and inside a
   // group all its CTAs longest first (pair c has about 2c + 2 key blocks).
@@ -415,9 +417,10 @@ cudaError_t tc_attention(const AttnArgs& a, cudaStream_t st) {
     if (ea != cudaSuccess) return ea;
   }
   dim3 grid(p.n_pairs * a.h * a.B);
-  attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmKV, tmKpe, p);
+  const cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(NTHREADS), SMEM_BYTES, st, tmQ,
+                                   tmKV, tmKpe, p);
   count_launches();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace mla

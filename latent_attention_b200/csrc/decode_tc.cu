@@ -162,6 +162,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_v = &abort_flag;
+  griddep_wait();
+  griddep_launch_dependents();
 
   const uint32_t rank = cluster_rank();
   const int u = blockIdx.x >> 1;
@@ -726,6 +728,8 @@ __global__ void __launch_bounds__(32 * HPB)
     combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                    __nv_bfloat16* __restrict__ o_lat, const int32_t* __restrict__ cu, int B,
                    int max_ctx, int h, int n_units, int min_len, uint32_t* status) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int hg = (h + HPB - 1) / HPB;
   const int b = blockIdx.x / hg;
   const int hh = (blockIdx.x % hg) * HPB + threadIdx.x / 32;
@@ -844,8 +848,10 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
       if (ea != cudaSuccess) return ea;
     }
     dim3 grid(2 * a.n_units, 1, (a.h + 127) / 128);
-    latent_attn_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(tmQ, tmQpe, tmC, tmCr, tmPO, tmOL, p);
+    e = launch_pdl(latent_attn_kernel, grid, dim3(NTHREADS), SMEM_BYTES, st, tmQ, tmQpe, tmC,
+                   tmCr, tmPO, tmOL, p);
     count_launches();
+    if (e != cudaSuccess) return e;
   }
   stage_event(2, st);
   // D3
@@ -853,16 +859,15 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st) {
   // times over (fewer, fuller blocks); one otherwise (few sequences, many
   // partial slots each, spread over as many SMs as possible)
   if ((int64_t)a.B * a.h >= 16LL * (2 * a.n_units)) {
-    combine_kernel<8><<<a.B * ((a.h + 7) / 8), 32 * 8, 0, st>>>(
-        a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B, a.max_ctx, a.h,
-        a.n_units, a.min_len, a.status);
+    e = launch_pdl(combine_kernel<8>, dim3(a.B * ((a.h + 7) / 8)), dim3(32 * 8), 0, st,
+                   (const float*)a.part_o, (const float*)a.part_lse, (__nv_bfloat16*)a.o_lat,
+                   a.cu_ctx, a.B, a.max_ctx, a.h, a.n_units, a.min_len, a.status);
   } else {
-    combine_kernel<1><<<a.B * a.h, 32, 0, st>>>(
-        a.part_o, a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B, a.max_ctx, a.h,
-        a.n_units, a.min_len, a.status);
+    e = launch_pdl(combine_kernel<1>, dim3(a.B * a.h), dim3(32), 0, st, (const float*)a.part_o,
+                   (const float*)a.part_lse, (__nv_bfloat16*)a.o_lat, a.cu_ctx, a.B,
+                   a.max_ctx, a.h, a.n_units, a.min_len, a.status);
   }
   count_launches();
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   stage_event(3, st);
   // D4: o[b, h, :] = o_lat[b, h, :] W_UV[h]^T  (per head: [B, R] x [R, dv])

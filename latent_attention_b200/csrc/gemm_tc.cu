@@ -238,6 +238,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   __syncthreads();
   tc_fence_after();
+  griddep_wait();               // the previous kernel's outputs (A, row scales) are ready
+  griddep_launch_dependents();
   const uint32_t tbase = tmem_base;
   const int nk = (p.K + BK - 1) / BK;
 
@@ -425,6 +427,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   // both CTAs' barriers exist before either addresses the other's
   cluster_sync_all();
   tc_fence_after();
+  griddep_wait();               // the previous kernel's outputs (A, row scales) are ready
+  griddep_launch_dependents();
   const uint32_t tbase = tmem_base;
   const int nk = (p.K + BK - 1) / BK;
   const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);       // the leader's
@@ -561,9 +565,10 @@ cudaError_t launch_single(int grid, const CUtensorMap& tmA, const CUtensorMap (&
   static std::atomic<uint64_t> smem_set{0};
   const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc_kernel<TBN, TST>, smem, smem_set);
   if (ea != cudaSuccess) return ea;
-  gemm_tc_kernel<TBN, TST><<<grid, NTHREADS, smem, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);
+  const cudaError_t e = launch_pdl(gemm_tc_kernel<TBN, TST>, dim3(grid), dim3(NTHREADS), smem, st,
+                                   tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);
   count_launches();
-  return cudaGetLastError();
+  return e;
 }
 
 template <int TBN2>
@@ -573,10 +578,10 @@ cudaError_t launch_pair(int pairs, const CUtensorMap& tmA, const CUtensorMap (&t
   static std::atomic<uint64_t> smem_set{0};
   const cudaError_t ea = set_dynamic_smem((const void*)gemm_tc2_kernel<TBN2>, smem, smem_set);
   if (ea != cudaSuccess) return ea;
-  gemm_tc2_kernel<TBN2><<<2 * pairs, NTHREADS, smem, st>>>(tmA, tmB[0], tmB[1], tmO[0], tmO[1],
-                                                            p);
+  const cudaError_t e = launch_pdl(gemm_tc2_kernel<TBN2>, dim3(2 * pairs), dim3(NTHREADS), smem,
+                                   st, tmA, tmB[0], tmB[1], tmO[0], tmO[1], p);
   count_launches();
-  return cudaGetLastError();
+  return e;
 }
 }  // namespace
 

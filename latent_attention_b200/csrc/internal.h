@@ -3,6 +3,7 @@
 
 #include <cstdint>
 #include <atomic>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -132,6 +133,26 @@ inline cudaError_t set_dynamic_smem(const void* kernel, int bytes,
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && bit) done_devices.fetch_or(bit, std::memory_order_release);
   return e;
+}
+
+// Launches a kernel with programmatic stream serialization: it may start
+// (prologue: barriers, TMEM, descriptor prefetch) while the previous kernel
+// of the stream finishes.  Only for kernels that call griddep_wait() first
+// (see sm100.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Launch accounting and stage events (defined in api.cu).

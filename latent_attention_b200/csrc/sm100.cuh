@@ -299,6 +299,20 @@ __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, ui
                : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream still
+// runs; griddep_wait() returns once that kernel has completed and its writes
+// are visible (at once when there is none), and every such kernel calls it
+// before it reads anything and before any thread exits, so a grid never
+// completes before the one it follows.  griddep_launch_dependents() lets the
+// next kernel of the stream start once every CTA of this one has called it.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
   asm volatile(
