@@ -50,7 +50,7 @@ constexpr int K_BYTES = 3 * BOX;                 // 48 KB per stage
 constexpr int V_BYTES = 2 * BOX;                 // 32 KB
 constexpr int OFF_Q = 0, OFF_K = 2 * Q_BYTES, OFF_V = OFF_K + K_BYTES;
 constexpr int SMEM_BYTES = OFF_V + 2 * V_BYTES + 1024;
-constexpr int NTHREADS = 640;
+constexpr int NTHREADS = 384;
 constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, DV, 0, 1);   // V is MN-major
 constexpr uint32_t TM_S = 0, TM_O = 256;                   // + 128 * tile
@@ -77,8 +77,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __shared__ __align__(8) uint64_t q_full, k_full, k_empty, v_full[2], v_empty[2], s_full[2],
       p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base;
-  __shared__ float mx_half[2][2][128];   // [tile][key half][row] block maxima
-  __shared__ float l_half[2][2][128];    // [tile][key half][row] final row sums
   __shared__ int abort_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -127,7 +125,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 8);          // both key halves' warps
+      mbar_init(&p_full[s], 4);          // the tile's softmax warps
       mbar_init(&pv_done[s], 1);
     }
     mbar_init(&k_full, 1);
@@ -240,13 +238,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp >= 4) {
-    // ---------------- softmax: two warpgroups per tile, one per half of the
-    // 128 keys of a block (warps 4-7 / 12-15 tile A, 8-11 / 16-19 tile B).
-    // The two halves of a row exchange their maxima through shared memory
-    // (named barrier 1 + tile), so both keep the same reference max; each
-    // keeps the row sum of its own keys.
-    const int x = ((warp - 4) >> 2) & 1;             // tile
-    const int hf = (warp - 4) >> 3;                  // key half: columns [64 hf, 64 hf + 64)
+    // ---------------- softmax: one warpgroup per tile (warps 4-7 tile A, 8-11
+    // tile B), thread = query row, all 128 keys of a block in one thread (no
+    // exchange between threads)
+    const int x = (warp - 4) >> 2;                   // tile
     const int quad = warp & 3;
     const int r = quad * 32 + lane;                  // query row within the tile
     const int qi = (x ? q0B : q0A) + r;              // query position
@@ -256,24 +251,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tO = tbase + lane_off + TM_O + x * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < my_nkv; ++j) {
+    for (int j = 0; ok && j < my_nkv; ++j) {
       // S_X(j) completion also implies PV_X(j-1) completion (in-order MMAs,
       // and S_X(j) was issued after PV_X(j-1) completed)
-      if (ok && !warp_wait(&s_full[x], j & 1, abort_v, p.status)) ok = false;
-      if (!ok) {   // after a failed wait: the halves' barriers stay paired
-        named_barrier_sync(1 + x, 256);
-        continue;
-      }
+      if (!warp_wait(&s_full[x], j & 1, abort_v, p.status)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tS + hf * 64, sr[0]);
-      tmem_ld32(tS + hf * 64 + 32, sr[1]);
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, sr[cc]);
       tmem_wait_ld();
       // Raw scores; the scale is folded into the exp argument below (scale > 0).
-      const int kmax = min(q_off + qi, Tk - 1) - j * BKV - hf * 64;  // last visible key here
-      if (kmax < 63) {
+      const int kmax = min(q_off + qi, Tk - 1) - j * BKV;   // last visible key here
+      if (kmax < BKV - 1) {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc)
+        for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (cc * 32 + i > kmax) sr[cc][i] = __float_as_uint(-INFINITY);
@@ -282,49 +273,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) mx4[k] = __uint_as_float(sr[0][k]);
 #pragma unroll
-      for (int i = 4; i < 64; i += 2)
+      for (int i = 4; i < 128; i += 2)
         mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], __uint_as_float(sr[i >> 5][i & 31]),
                                   __uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]));
-      // combine with the other half of the row; after this barrier both halves
-      // have loaded S, so P may be written over it
-      mx_half[x][hf][r] = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
-      named_barrier_sync(1 + x, 256);
-      const float mrow = fmaxf(mx_half[x][0][r], mx_half[x][1][r]);
-      const float mx = fmaxf(m_ref, p.scale_log2 * mrow);
+      const float mx =
+          fmaxf(m_ref, p.scale_log2 * max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])));
       const bool grow = mx > m_ref + kRescaleLog2;    // also true for the first block
       const float alpha = grow ? ex2(m_ref - mx) : 1.f;
       if (grow) {
         l *= alpha;
         m_ref = mx;
       }
-      // P = 2^(scale * s - m_ref) as bf16 pairs: this half's 64 keys go to
-      // columns [32 hf, 32 hf + 32) of S
+      // P = 2^(scale * s - m_ref) as bf16 pairs over the first 64 columns of S,
+      // 16 columns (32 keys) at a time: P of keys [32q, 32q + 32) goes over
+      // the scores of keys [16q, 16q + 16), which are already used
       float ls[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
       const float sc = p.scale_log2;
-      uint32_t w[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int i = 2 * e;
-        const float p0 = ex2(fmaf(__uint_as_float(sr[i >> 5][i & 31]), sc, -m_ref));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[(i + 1) >> 5][(i + 1) & 31]), sc, -m_ref));
-        ls[e & 7] += p0 + p1;
-        w[e] = pack_bf16(p0, p1);
+      for (int q = 0; q < 4; ++q) {
+        uint32_t wv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[q][2 * e]), sc, -m_ref));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[q][2 * e + 1]), sc, -m_ref));
+          ls[e & 7] += p0 + p1;
+          wv[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + q * 16, wv);
       }
-      tmem_st32(tS + hf * 32, w);
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_X holds the sum through block j-1 (complete, see above); each half
-        // rescales its 64 of the 128 value columns
+        // O_X holds the sum through block j-1 (complete, see above)
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tO + hf * 64 + cc * 32, o);
+          tmem_ld32(tO + cc * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + hf * 64 + cc * 32, o);
+          tmem_st32(tO + cc * 32, o);
         }
       }
       tmem_wait_st();
@@ -332,20 +321,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    // row sum of both halves (each half passes my_nkv + 1 barriers on every
-    // path)
-    l_half[x][hf][r] = l;
-    named_barrier_sync(1 + x, 256);
-    l = l_half[x][0][r] + l_half[x][1][r];
     if (ok && my_nkv > 0 && warp_wait(&pv_done[x], (my_nkv - 1) & 1, abort_v, p.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const bool row_ok = qi < Tq;
-      __nv_bfloat16* dst = p.o + ((int64_t)(row0 + qi) * p.h + hh) * DV + hf * 64;
+      __nv_bfloat16* dst = p.o + ((int64_t)(row0 + qi) * p.h + hh) * DV;
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        tmem_ld32(tO + hf * 64 + cc * 32, o);
+        tmem_ld32(tO + cc * 32, o);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
