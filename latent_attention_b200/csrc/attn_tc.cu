@@ -16,7 +16,7 @@
 // loads serves both tiles.  The CTAs of eight (sequence, head) pairs at a
 // time run together, longest first, so a head's keys and values leave HBM
 // once and the grid ends on short CTAs.  Warp roles
-// (640 threads):
+// (384 threads):
 //   warp 0       TMA: Q of both tiles (once), K (one stage of 3 boxes)
 //   warp 2       TMA: V ring (2 stages of 2 boxes of 64 value columns)
 //   warp 1       TMEM allocation and MMA issue, in the order
@@ -24,9 +24,9 @@
 //                so that the tensor core works on one tile while the other
 //                tile's softmax runs; S_X(j+1) follows PV_X(j) in issue order,
 //                which is execution order (P_X(j) lives in S_X's columns).
-//   warps 4-7 / 12-15  softmax of tile A, keys 0-63 / 64-127 of each block;
-//   warps 8-11 / 16-19 the same for tile B (thread = query row and key half;
-//                the halves of a row exchange maxima through shared memory):
+//   warps 4-7    softmax of tile A, warps 8-11 of tile B (thread = query
+//                row, all 128 keys of a block in one thread, so no exchange
+//                between threads; 12 warps leave each thread 168 registers):
 //                S from TMEM, causal mask on the diagonal block,
 //                running max with lazy rescaling (O and l rescaled only when
 //                the max grows by more than 2^8), P as bf16 pairs written
